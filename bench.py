@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA / HCA compressed-attention hot path on B200.
+
+Headline (the `value` of the JSON line): CSA decode queries/s at 128K context --
+32 sequences x 1 new query each, 32768 compressed entries per sequence, top-k 1024,
+window 128, 64 heads of dim 512, MXFP4 indexer with 64 heads of dim 128.  One step
+= MXFP4 encoding of the indexer queries, indexer scores over every entry, top-k
+selection, sparse MQA over the selected entries plus the window.  The cache is
+resident in HBM; 4 independent input replicas rotate between steps so that every
+step reads inputs that are not in the 126 MB L2.
+
+Also reported in the same line: CSA prefill T=8192 tokens/s and HCA prefill
+T=65536 tokens/s, each with the roofline of its dominant kernel; end-to-end decode
+through the public API with host buffers; the CPU oracle on a bounded sample.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+For N > 1 launch one process per GPU (torchrun); every rank runs its own 32
+sequences (weak scaling, no collective on the data path); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "CSA decode queries/s at 128K ctx; prefill tok/s; % of HBM / tensor roofline"
+UNIT = "queries/s"
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                       "-i", str(self.gpu), "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.p.terminate()
+        self.p.wait()
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        top = max(sm)
+        loaded = [x for x in sm if x >= 0.5 * top] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- distributed
+class Dist:
+    def __init__(self):
+        import torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if torch.cuda.is_available():
+            torch.cuda.set_device(self.local_rank)
+        if self.world > 1:
+            import torch.distributed as dist
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=180))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if self.pg is None:
+            return x
+        import torch
+        dev = torch.device("cuda", self.local_rank) if torch.cuda.is_available() else torch.device("cpu")
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- decode 128K
+def decode_bytes_per_query(wl) -> dict:
+    """Algorithmic bytes of one decode query (compulsory traffic, no scratch)."""
+    E, k, W, D, H, Hi, Di = wl.E, wl.k, wl.W, wl.D, wl.H, wl.Hi, wl.Di
+    keys = E * (Di // 2 + Di // 32)
+    qi = Hi * (Di * 4) + Hi * 4           # raw fp32 indexer query + head weights
+    q_fp4 = Hi * (Di // 2 + Di // 32)
+    gathered = k * D * 2
+    window = W * D * 2
+    q_o = 2 * H * D * 2
+    idx = k * 4
+    score_out = E * 4
+    return {"step": keys + qi + gathered + window + q_o + idx,
+            "index_score": keys + q_fp4 + Hi * 4 + score_out,
+            "attention": gathered + window + q_o + idx,
+            "keys": keys}
+
+
+def setup_decode(wl, dev, replicas: int):
+    import torch
+    from compressed_sparse_long_02_b200 import binding as B
+    from compressed_sparse_long_02_b200 import synth
+    caches, steps = [], []
+    for r in range(replicas):
+        d = synth.decode_inputs_torch(wl, dev, replica=r)
+        k_fp4, k_sc = B.csa_quantize_mxfp4(d["ki"])
+        del d["ki"]
+        Bn = d["q"].shape[0]
+        caches.append({"entries": d["entries"], "k_fp4": k_fp4, "k_scale": k_sc, "window": d["window"],
+                       "window_base": (d["pos"] - wl.W + 1).to(torch.int32),
+                       "n_entries": torch.full((Bn,), wl.E, dtype=torch.int32, device=dev)})
+        steps.append({"q": d["q"], "qi": d["qi"], "w": d["w"], "pos": d["pos"]})
+    torch.cuda.synchronize()
+    Bn = wl.B
+    ws = {
+        "q_fp4": torch.empty((Bn, wl.Hi, wl.Di // 2), dtype=torch.uint8, device=dev),
+        "q_scale": torch.empty((Bn, wl.Hi, wl.Di // 32), dtype=torch.uint8, device=dev),
+        "scores": torch.empty((Bn, wl.E), dtype=torch.float32, device=dev),
+        "idx": torch.empty((Bn, wl.k), dtype=torch.int32, device=dev),
+        "cnt": torch.empty((Bn,), dtype=torch.int32, device=dev),
+        "seq": torch.arange(Bn, dtype=torch.int32, device=dev),
+        "attn_ws": torch.empty(B.csa_sparse_attn_workspace(Bn, wl.H, wl.D, wl.k, wl.W), dtype=torch.uint8,
+                               device=dev),
+        "out": torch.empty((Bn, wl.H, wl.D), dtype=torch.bfloat16, device=dev),
+    }
+    return caches, steps, ws
+
+
+def decode_step(wl, cache, step, ws, ev=None):
+    """One decode step as four C-ABI calls; `ev` (optional) gets CUDA events between calls."""
+    from compressed_sparse_long_02_b200 import binding as B
+    if ev is not None:
+        ev[0].record()
+    B.csa_quantize_mxfp4(step["qi"], ws["q_fp4"], ws["q_scale"])
+    if ev is not None:
+        ev[1].record()
+    B.csa_index_score(ws["q_fp4"], ws["q_scale"], step["w"], step["pos"], ws["seq"], cache["k_fp4"],
+                      cache["k_scale"], cache["n_entries"], m=wl.m, scores=ws["scores"])
+    if ev is not None:
+        ev[2].record()
+    B.csa_topk_select(ws["scores"], step["pos"], ws["seq"], cache["n_entries"], k=wl.k, m=wl.m, E_max=wl.E,
+                      idx=ws["idx"], cnt=ws["cnt"])
+    if ev is not None:
+        ev[3].record()
+    B.csa_sparse_attn(step["q"], step["pos"], ws["seq"], cache["entries"], ws["idx"], ws["cnt"], cache["window"],
+                      cache["window_base"], W=wl.W, out=ws["out"], workspace=ws["attn_ws"])
+    if ev is not None:
+        ev[4].record()
+
+
+def bench_decode(args, dist, peaks):
+    import torch
+    from compressed_sparse_long_02_b200 import binding as B
+    from compressed_sparse_long_02_b200 import synth
+    wl = synth.WORKLOADS["csa_decode_128k"]
+    dev = torch.device("cuda", dist.local_rank)
+    R = args.replicas
+    caches, steps, ws = setup_decode(wl, dev, R)
+    for i in range(args.warmup):
+        decode_step(wl, caches[i % R], steps[i % R], ws)
+    torch.cuda.synchronize()
+    assert B.csa_get_device_error() == 0, "device error during warm-up"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dist.local_rank)
+    clocks.start()
+    dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(args.steps):
+        decode_step(wl, caches[i % R], steps[i % R], ws, evs[i])
+    end.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    ms_local = start.elapsed_time(end)
+    ms = dist.max(ms_local)
+    assert B.csa_get_device_error() == 0, "device error in the timed region"
+
+    per = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in
+           enumerate(["quantize", "index_score", "topk_select", "attention"])}
+    nb = decode_bytes_per_query(wl)
+    queries_per_step = wl.B * dist.world
+    value = queries_per_step * args.steps / (ms / 1e3)
+    ms_step = ms / args.steps
+    dom = max(per, key=per.get)
+    dom_bytes = {"index_score": nb["index_score"], "attention": nb["attention"],
+                 "quantize": wl.Hi * wl.Di * 4, "topk_select": wl.E * 4}[dom] * wl.B
+    achieved = dom_bytes / (per[dom] / 1e3) / 1e9
+    step_gbs = nb["step"] * wl.B / (ms_local / args.steps / 1e3) / 1e9
+    res = {
+        "value": value, "ms_per_step": ms_step,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                     "algorithmic_bytes_per_launch": dom_bytes, "peak_source": peaks["source"]},
+        "step_roofline": {"bound": "hbm", "algorithmic_bytes": nb["step"] * wl.B, "achieved_gbs": round(step_gbs, 1),
+                          "frac": round(step_gbs / peaks["hbm_gbs"], 4)},
+        "per_call_us": {k: round(v * 1e3, 2) for k, v in per.items()},
+        "clocks": clk,
+        "gpu_launches": args.steps * 5,  # quantize, index score, top-k, attention, split merge
+    }
+    res["e2e"] = bench_decode_e2e(args, wl, caches, steps, ws, dist)
+    del caches, steps, ws
+    torch.cuda.empty_cache()
+    return wl, res
+
+
+def bench_decode_e2e(args, wl, caches, steps, ws, dist):
+    """Decode through the public API with host buffers: pinned H2D of the step's inputs
+    (q, indexer query, head weights, positions) and D2H of the output, every step."""
+    import torch
+    from compressed_sparse_long_02_b200 import layer
+    R = len(caches)
+    host = []
+    for r in range(R):
+        host.append({k: v.cpu().pin_memory() for k, v in steps[r].items()})
+    dev_in = {k: torch.empty_like(v) for k, v in steps[0].items()}
+    out_host = torch.empty((wl.B, wl.H, wl.D), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host[0].values())
+    d2h = out_host.numel() * out_host.element_size()
+    lws = {"q_fp4": ws["q_fp4"], "q_scale": ws["q_scale"], "idx": ws["idx"], "cnt": ws["cnt"], "seq": ws["seq"],
+           "attn_ws": ws["attn_ws"],
+           "index_ws": torch.empty(layer.B.csa_index_topk_workspace(wl.B, wl.E, wl.k), dtype=torch.uint8,
+                                   device=ws["out"].device)}
+
+    def one(i):
+        src = host[i % R]
+        for k in dev_in:
+            dev_in[k].copy_(src[k], non_blocking=True)
+        r = layer.csa_decode(wl, caches[i % R], dev_in, lws, out=ws["out"])
+        out_host.copy_(r["out"], non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for i in range(args.warmup):
+        one(i)
+    dist.barrier()
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(i)
+    t = dist.max(time.perf_counter() - t0)
+    return {"value": wl.B * dist.world * args.steps / t, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+# ----------------------------------------------------------------------------- prefill
+def _dev_inputs(inp, dev):
+    import numpy as np
+    import torch
+    out = {}
+    for k, v in inp.items():
+        if v.dtype == np.uint16:
+            out[k] = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev)
+        else:
+            out[k] = torch.from_numpy(np.ascontiguousarray(v)).to(dev)
+    return out
+
+
+def bench_prefill(name, steps, warmup, dist, peaks):
+    import torch
+    from compressed_sparse_long_02_b200 import binding as B
+    from compressed_sparse_long_02_b200 import layer, synth
+    wl = synth.WORKLOADS[name]
+    dev = torch.device("cuda", dist.local_rank)
+    t = synth.prefill_inputs_torch(wl, dev)
+    run = layer.csa_prefill if wl.kind == "csa_prefill" else layer.hca_prefill
+    for _ in range(warmup):
+        run(wl, t)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    s.record()
+    for _ in range(steps):
+        run(wl, t)
+    e.record()
+    torch.cuda.synchronize()
+    ms = dist.max(s.elapsed_time(e)) / steps
+    assert B.csa_get_device_error() == 0
+    # dominant kernel: the attention call, timed alone on the same inputs
+    r = run(wl, t)
+    torch.cuda.synchronize()
+    seq = torch.zeros(wl.T, dtype=torch.int32, device=dev)
+    pos = torch.arange(wl.T, dtype=torch.int32, device=dev)
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    ne = torch.tensor([wl.E], dtype=torch.int32, device=dev)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(1, steps)
+    a0.record()
+    for _ in range(reps):
+        if wl.kind == "csa_prefill":
+            B.csa_sparse_attn(r["q"], pos, seq, r["entries"], r["idx"], r["cnt"], r["window"], zero, W=wl.W,
+                              out=r["out"])
+        else:
+            B.hca_attn(r["q"], pos, seq, r["entries"], ne, r["window"], zero, mprime=wl.m, W=wl.W, out=r["out"])
+    a1.record()
+    torch.cuda.synchronize()
+    attn_ms = a0.elapsed_time(a1) / reps
+    flops = attention_flops(wl)
+    tf = flops / (attn_ms / 1e3) / 1e12
+    out = {"workload": name, "tokens": wl.T, "tok_per_s": wl.T * dist.world / (ms / 1e3), "ms_per_step": ms,
+           "roofline": {"bound": "tensor", "kernel": "attention", "achieved": round(tf, 1),
+                        "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                        "frac": round(tf / peaks["bf16_tflops_sustained"], 4), "attention_ms": round(attn_ms, 4),
+                        "algorithmic_flops": flops}}
+    del t, r
+    torch.cuda.empty_cache()
+    return out
+
+
+def attention_flops(wl) -> float:
+    """2 x (QK + PV) x H x D over every (query, key) pair the layer attends to."""
+    tot = 0
+    for t in range(wl.T):
+        nv = (t + 1) // wl.m
+        sel = min(wl.k, nv) if wl.kind == "csa_prefill" else min(nv, wl.E)
+        tot += sel + min(wl.W, t + 1)
+    return 4.0 * wl.H * wl.D * tot
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_oracle_decode(wl, n_seq: int, budget_s: float = 20.0, seed_replica: int = 0):
+    """The oracle on a bounded sample of decode queries (full 32768-entry caches)."""
+    import numpy as np
+    import oracle
+    from compressed_sparse_long_02_b200 import synth
+    d = synth.decode_inputs(wl, B=n_seq, seed_offset=seed_replica)
+    kp, ks = oracle.mxfp4_quantize(d["ki"])
+    done, t_used = 0, 0.0
+    cores = os.cpu_count() or 1
+    chunk = max(1, min(n_seq, cores))
+    while done < n_seq and t_used < budget_s:
+        seqs = np.arange(done, min(n_seq, done + chunk))
+        t0 = time.perf_counter()
+        qp, qs = oracle.mxfp4_quantize(d["qi"][seqs])
+        qpf = np.zeros((n_seq,) + qp.shape[1:], np.uint8)
+        qsf = np.zeros((n_seq,) + qs.shape[1:], np.uint8)
+        qpf[seqs], qsf[seqs] = qp, qs
+        oracle.csa_decode(wl, d["entries"], kp, ks, d["q"], qpf, qsf, d["w"], d["window"], d["pos"], seqs=seqs)
+        t_used += time.perf_counter() - t0
+        done += len(seqs)
+    threads = int(os.environ.get("OMP_NUM_THREADS", cores))
+    return {"value": done / t_used, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{done} decode queries (full {wl.E}-entry caches, k={wl.k}, W={wl.W}) in {t_used:.1f} s"}
+
+
+def run_reference(args, dist):
+    """The reference arm: the CPU oracle, as it stands, on bounded decode samples."""
+    if dist.rank != 0:
+        return None
+    from compressed_sparse_long_02_b200 import synth
+    wl = synth.WORKLOADS["csa_decode_128k"]
+    cores = os.cpu_count() or 1
+    per_step = max(1, min(wl.B, cores))
+    import numpy as np
+    import oracle
+    d = synth.decode_inputs(wl, B=per_step)
+    kp, ks = oracle.mxfp4_quantize(d["ki"])
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        qp, qs = oracle.mxfp4_quantize(d["qi"])
+        oracle.csa_decode(wl, d["entries"], kp, ks, d["q"], qp, qs, d["w"], d["window"], d["pos"])
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = per_step * len(times) / tot
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": decode_config(wl, args),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(os.environ.get("OMP_NUM_THREADS", cores)),
+                             "kind": "oracle",
+                             "sample": f"{per_step} decode queries per step (full {wl.E}-entry caches)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return line
+
+
+def decode_config(wl, args):
+    return {"workload": "csa_decode_128k", "sequences_per_gpu": wl.B, "context": wl.L, "entries": wl.E,
+            "top_k": wl.k, "window": wl.W, "heads": wl.H, "head_dim": wl.D, "indexer_heads": wl.Hi,
+            "indexer_dim": wl.Di, "indexer_format": "MXFP4 (E2M1, UE8M0 per 32)", "parallelism": f"dp{args.gpus}",
+            "l2": f"inputs larger than L2: {args.replicas} rotating input replicas (~1.1 GB each); a replica is "
+                  f"re-read only after {args.replicas - 1} other steps"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="csa", choices=["csa", "reference"])
+    ap.add_argument("--replicas", type=int, default=4)
+    ap.add_argument("--no-secondary", action="store_true", help="skip the prefill lines")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    dist = Dist()
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, dist)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+            return
+        import torch
+        from compressed_sparse_long_02_b200 import binding
+        binding.lib()
+        peaks = load_peaks()
+        wl, res = bench_decode(args, dist, peaks)
+        line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16+mxfp4 (fp32 accumulate)",
+                "data": "synthetic (seeded; N(0,1) caches and queries, U(0,1) head weights)",
+                "config": decode_config(wl, args), "roofline": res["roofline"],
+                "step_roofline": res["step_roofline"], "per_call_us": res["per_call_us"], "e2e": res["e2e"],
+                "clocks": res["clocks"], "gpu_launches": res["gpu_launches"]}
+        if not args.no_secondary:
+            sec_steps = 5
+            line["prefill"] = bench_prefill("csa_prefill_8k", sec_steps, 2, dist, peaks)
+            line["hca_prefill"] = bench_prefill("hca_prefill_64k", 3, 1, dist, peaks)
+        if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
+            line["cpu_baseline"] = cpu_oracle_decode(wl, n_seq=min(wl.B, max(4, os.cpu_count() or 4)))
+        if dist.rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

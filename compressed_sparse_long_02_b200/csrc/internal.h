@@ -1,0 +1,115 @@
+// internal.h -- host-side declarations shared by the library's translation units.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "csa.h"
+
+namespace csa {
+
+// device error word of the current device (lazily resolved, cached per device)
+int32_t* device_error_word();
+int num_sms();
+
+// Raise `fn`'s dynamic shared-memory limit to `bytes` on the current device (once per
+// size; `cache` holds the limit already set, one slot per device).
+inline cudaError_t set_dyn_smem(const void* fn, size_t bytes, int* cache) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (cache[dev] >= static_cast<int>(bytes)) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess) cache[dev] = static_cast<int>(bytes);
+  return e;
+}
+
+// ---------------------------------------------------------------- compressor / norm / rope
+struct NormRopeArgs {
+  const void* x;
+  int in_bf16;
+  int64_t rows;
+  int heads;
+  int C;
+  const int32_t* pos;  // nullable
+  int64_t pos_mod;
+  int norm;
+  float eps;
+  int rope_dims;
+  float theta;
+  uint16_t* out;
+};
+cudaError_t launch_norm_rope(const NormRopeArgs& a, cudaStream_t s);
+
+struct PoolArgs {
+  const void* kv;
+  const void* logits;
+  int in_bf16;
+  const float* bias;
+  int B, T, C, m, overlap;
+  int norm;
+  float eps;
+  int rope_dims;
+  float theta;
+  uint16_t* entries;  // nullable, [B, E_max, C]
+  int E_max;
+  uint8_t* fp4;       // nullable, [B, E_max, C/2]
+  uint8_t* fp4_scale; // nullable, [B, E_max, C/32]
+};
+cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- MXFP4
+cudaError_t launch_quantize_mxfp4(const void* x, int in_bf16, int64_t rows, int cols, uint8_t* packed,
+                                  uint8_t* scales, cudaStream_t s);
+
+// ---------------------------------------------------------------- indexer + top-k
+struct IndexArgs {
+  int Nq, Hi, Di, k, m, B, E_max;
+  const uint8_t* q_fp4;
+  const uint8_t* q_scale;
+  const float* w;
+  const int32_t* q_pos;
+  const int32_t* q_seq;
+  const uint8_t* k_fp4;
+  const uint8_t* k_scale;
+  const int32_t* n_entries;
+  int32_t* idx_out;
+  int32_t* cnt_out;
+  float* score_out;  // nullable
+  float* scores_ws;  // [Nq, E_stride]
+  int E_stride;
+};
+size_t index_workspace_bytes(int Nq, int E_max, int k);
+cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s);  // writes scores_ws (+ score_out)
+cudaError_t launch_topk_select(const IndexArgs& a, cudaStream_t s);  // reads scores_ws
+inline cudaError_t launch_index_topk(const IndexArgs& a, cudaStream_t s) {
+  const cudaError_t e = launch_index_score(a, s);
+  return e != cudaSuccess ? e : launch_topk_select(a, s);
+}
+
+// ---------------------------------------------------------------- attention
+struct AttnArgs {
+  int Nq, H, D, k, W;
+  float scale;
+  const uint16_t* q;
+  const int32_t* q_pos;
+  const int32_t* q_seq;
+  int B, E_max;
+  const uint16_t* entries;
+  const int32_t* idx;       // sparse mode; nullptr in dense (HCA) mode
+  const int32_t* cnt;       // sparse mode
+  const int32_t* n_entries; // dense mode
+  int dense;                // 1: every visible entry (HCA); 0: the idx/cnt selection
+  int mprime;               // dense mode
+  int Tw;
+  const uint16_t* window;
+  const int32_t* window_base;
+  uint16_t* out;
+  float* lse;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t attn_workspace_bytes(int Nq, int H, int D, int max_keys);
+cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s);
+
+}  // namespace csa

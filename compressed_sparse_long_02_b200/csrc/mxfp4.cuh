@@ -1,0 +1,50 @@
+// mxfp4.cuh -- MXFP4 (E2M1 codes, UE8M0 scale per 32 elements) encoding on the device.
+//
+// Rule (the lightning indexer runs in FP4 -- dev.to "How DeepSeek-V4 Achieves
+// Million-Token Contexts ...", section "Two Compression Strategies: CSA and HCA"):
+//   E    = smallest integer with amax <= 6 * 2^E, clamped to [-127, 127]; amax == 0 -> -127
+//   code = round-half-even of x / 2^E onto {0, .5, 1, 1.5, 2, 3, 4, 6}; bit 3 = sign of x
+//   scale byte = E + 127; element 2i in the low nibble of byte i.
+// Every step is exact (power-of-two scaling, comparisons), so the bytes are a pure
+// function of the input bits.
+#pragma once
+#include <cstdint>
+
+namespace csa {
+
+// smallest E with amax <= 6 * 2^E: write amax = f * 2^k, f in [1,2); 6 * 2^E = 1.5 * 2^(E+2),
+// so E = k - 2 when f <= 1.5 and k - 1 otherwise.
+__device__ __forceinline__ int mx_block_exponent(float amax) {
+  if (!(amax > 0.f)) return -127;
+  const uint32_t bits = __float_as_uint(amax);
+  const int ef = static_cast<int>((bits >> 23) & 0xFFu);
+  if (ef == 0) return -127;  // subnormal amax < 2^-126 <= 6 * 2^-127
+  int E = ef - 129 + ((bits & 0x7FFFFFu) > 0x400000u ? 1 : 0);
+  return E < -127 ? -127 : (E > 127 ? 127 : E);
+}
+
+__device__ __forceinline__ uint32_t e2m1_code(float x, int E) {
+  const float a = fabsf(ldexpf(x, -E));
+  const uint32_t c = a <= 0.25f   ? 0u
+                     : a < 0.75f  ? 1u
+                     : a <= 1.25f ? 2u
+                     : a < 1.75f  ? 3u
+                     : a <= 2.5f  ? 4u
+                     : a < 3.5f   ? 5u
+                     : a <= 5.0f  ? 6u
+                                  : 7u;
+  return c | (signbit(x) ? 8u : 0u);
+}
+
+// Encode the pair (x0, x1) held by this thread, where 16 consecutive lanes (aligned
+// to 16) hold one 32-element block.  All 32 lanes of the warp must call it.
+__device__ __forceinline__ void mxfp4_encode_pair(float x0, float x1, uint8_t& byte, uint8_t& scale_byte) {
+  float am = fmaxf(fabsf(x0), fabsf(x1));
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  const int E = mx_block_exponent(am);
+  byte = static_cast<uint8_t>(e2m1_code(x0, E) | (e2m1_code(x1, E) << 4));
+  scale_byte = static_cast<uint8_t>(E + 127);
+}
+
+}  // namespace csa

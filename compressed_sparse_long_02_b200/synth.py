@@ -27,8 +27,8 @@ import math
 
 import numpy as np
 
-__all__ = ["Workload", "WORKLOADS", "prefill_inputs", "decode_inputs", "decode_inputs_torch",
-           "to_dtype_np"]
+__all__ = ["Workload", "WORKLOADS", "prefill_inputs", "prefill_inputs_torch", "decode_inputs",
+           "decode_inputs_torch", "to_dtype_np"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -135,6 +135,31 @@ def prefill_inputs(wl: Workload, T: int | None = None, B: int | None = None) -> 
         out["zi"] = to_dtype_np(_normal(rng, (B, T, Di)), wl.dtype)
         out["bias_i"] = _normal(rng, (wl.slots, Di), wl.bias_var).astype(np.float32)
         out["w"] = rng.uniform(0.0, 1.0, (B, T, Hi)).astype(np.float32)
+    return out
+
+
+def prefill_inputs_torch(wl: Workload, device, T: int | None = None, replica: int = 0) -> dict:
+    """Prefill inputs drawn directly on ``device`` (same keys, shapes and distributions as
+    :func:`prefill_inputs`, torch dtypes) for the workloads too large to draw on the host."""
+    import torch
+    T = wl.T if T is None else T
+    g = torch.Generator(device=device)
+    g.manual_seed(wl.seed * 7919 + 17 + replica)
+    act = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+
+    def nrm(shape, var=1.0):
+        return (torch.randn(shape, generator=g, device=device, dtype=torch.float32) * math.sqrt(var)).to(act)
+
+    C, H = wl.C, wl.H
+    out = {"kv": nrm((1, T, C)), "z": nrm((1, T, C)),
+           "bias": torch.randn((wl.slots, C), generator=g, device=device) * math.sqrt(wl.bias_var),
+           "q": nrm((1, T, H, C), wl.q_var)}
+    if wl.kind == "csa_prefill":
+        out["qi"] = nrm((1, T, wl.Hi, wl.Di))
+        out["ki"] = nrm((1, T, wl.Di))
+        out["zi"] = nrm((1, T, wl.Di))
+        out["bias_i"] = torch.randn((wl.slots, wl.Di), generator=g, device=device) * math.sqrt(wl.bias_var)
+        out["w"] = torch.rand((1, T, wl.Hi), generator=g, device=device)
     return out
 
 

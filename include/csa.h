@@ -1,0 +1,231 @@
+/*
+ * csa.h -- C ABI of libcsa.so: CSA / HCA compressed attention on NVIDIA B200 (sm_100a).
+ *
+ * The layer (pages: "DeepSeek-V4: Million-Token Context" explainer, CSA and HCA
+ * stages; "Follow the white rabbit: DeepSeek V4's architecture in 3D", CSA / HCA /
+ * window / indexer paragraphs; "DeepSeek-V4: Towards Highly Efficient
+ * Million-Token Context Intelligence" summary, section 2.3):
+ *
+ *   csa_compress        every m tokens -> one KV entry by per-channel softmax pooling
+ *                       (CSA: m = 4, each entry also pools the previous group of 4;
+ *                       HCA: m' = 128, no overlap), then RMSNorm and partial RoPE.
+ *   csa_norm_rope       RMSNorm + partial RoPE of query heads (and raw window rows).
+ *   csa_quantize_mxfp4  FP4 (E2M1, UE8M0 scale per 32) encoding for the lightning indexer.
+ *   csa_index_topk      lightning-indexer scores of every visible entry, then top-k.
+ *   csa_sparse_attn     shared-KV MQA over the top-k entries plus the raw-token window.
+ *   hca_attn            shared-KV MQA over every visible HCA entry plus the window.
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers unless marked "host".  The caller
+ *     owns every buffer; the library allocates nothing on these calls and keeps
+ *     only one lazily created 4-byte device error word per device.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Only argument validation is synchronous.  Results are ready when
+ *     the stream reaches the call.
+ *   - Return codes only: nothing is printed, nothing aborts.  Invalid shapes
+ *     give CSA_ERR_INVALID_ARG, shapes outside the supported set
+ *     CSA_ERR_UNSUPPORTED, pointers that are not 16-byte aligned
+ *     CSA_ERR_ALIGNMENT, a workspace that is too small CSA_ERR_WORKSPACE, a
+ *     failed launch CSA_ERR_CUDA.  Faults detected on the device (an index out of
+ *     range, a wait that ran out of time) are recorded in the device error word,
+ *     read with csa_get_device_error.
+ *   - bf16 is IEEE bfloat16 stored as uint16_t; row-major, innermost index last.
+ *   - Positions are absolute token positions.  Entry j of a sequence covers
+ *     tokens [m*j, m*j+m-1] and sits at position m*(j+1)-1, so a query at
+ *     position t sees entries j < floor((t+1)/m): a group is usable once complete;
+ *     the window covers the unfinished one.
+ */
+#ifndef CSA_H
+#define CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#ifndef __CUDA_RUNTIME_H__
+typedef struct CUstream_st* cudaStream_t;
+#endif
+
+#if defined(__GNUC__)
+#define CSA_API __attribute__((visibility("default")))
+#else
+#define CSA_API
+#endif
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1,
+  CSA_ERR_ALIGNMENT = 2,
+  CSA_ERR_UNSUPPORTED = 3,
+  CSA_ERR_WORKSPACE = 4,
+  CSA_ERR_CUDA = 5,
+  CSA_ERR_DEVICE = 6
+} csa_status;
+
+typedef enum { CSA_F32 = 0, CSA_BF16 = 1 } csa_dtype;
+
+/* device error word values (csa_get_device_error) */
+#define CSA_DEVERR_NONE 0
+#define CSA_DEVERR_TIMEOUT 1   /* a pipeline wait exceeded its bound; the kernel returned early */
+#define CSA_DEVERR_INDEX 2     /* an entry index was outside [0, visible entries) and was skipped */
+
+
+/* Pooling configuration.  CSA: m = 4, overlap = 1; HCA: m = 128, overlap = 0. */
+typedef struct {
+  int m;            /* tokens per entry, 1..128 */
+  int overlap;      /* 1: entry j also pools group j-1 (slots 0..m-1), own group in slots m..2m-1 */
+  int C;            /* channels; multiple of 64, at most 1024 */
+  int norm;         /* 1: RMSNorm (unit gain) of entries before RoPE */
+  float eps;        /* RMSNorm epsilon */
+  int rope_dims;    /* partial RoPE on the last rope_dims channels (even, <= C; 0 = none) */
+  float rope_theta; /* RoPE base */
+  csa_dtype in_dtype;
+} csa_pool_cfg;
+
+/*
+ * csa_compress -- softmax-weighted pooling of raw KV into compressed entries.
+ * ("DeepSeek-V4: Million-Token Context", CSA stage: every m=4 tokens become one
+ * entry through a learned softmax weighting; "Follow the white rabbit", CSA
+ * paragraph: each entry also draws on the previous group of four; HCA
+ * paragraph: weighted averages of 128 tokens with different weights for
+ * different parts of the representation, i.e. per channel.)
+ *
+ *   a[s,c]   = logits[tok_s, c] + slot_bias[s, c]
+ *   e[j,c]   = sum_s softmax_s(a[., c])[s] * kv[tok_s, c]   (slots of group j-1 absent for j = 0)
+ *   entries  = RoPE_{m(j+1)-1}(RMSNorm(e[j]))  (norm / RoPE per cfg), stored bf16
+ *
+ * B sequences of T tokens each (kv, logits: [B, T, C], element type cfg->in_dtype);
+ * slot_bias: float32 [(1+overlap)*m, C].
+ * entries (bf16 [B, E_max, C], may be NULL): entry j of sequence b for j < floor(T/m);
+ *   E_max >= floor(T/m).
+ * fp4_out / fp4_scale (may be NULL; both or neither): the pooled entries before
+ *   norm and RoPE, MXFP4-encoded as in csa_quantize_mxfp4: [B, E_max, C/2] and
+ *   [B, E_max, C/32] bytes (the lightning indexer's key cache).
+ * window_kv (bf16 [B, T, C], may be NULL): raw-token rows RoPE_u(RMSNorm(kv[u])) used
+ *   by the sliding window ("Follow the white rabbit": the most recent 128 tokens
+ *   kept separately).
+ * Errors: INVALID_ARG for T < 0, B < 1, m outside 1..128, odd rope_dims;
+ * UNSUPPORTED for C not a multiple of 64 or > 1024 (fp4 output needs C % 32 == 0).
+ */
+CSA_API csa_status csa_compress(const csa_pool_cfg* cfg, int B, int T, const void* kv, const void* logits,
+                        const float* slot_bias, void* entries, int E_max, uint8_t* fp4_out,
+                        uint8_t* fp4_scale, void* window_kv, cudaStream_t stream);
+
+/*
+ * csa_norm_rope -- RMSNorm (unit gain) and partial RoPE of `heads` vectors per row
+ * ("DeepSeek-V4: Towards Highly Efficient ...", section 2.3 "Other details": RMSNorm
+ * on query heads and KV entries right before core attention; dev.to "How DeepSeek-V4
+ * Achieves ...": partial rotary positional embedding).
+ * x: [rows, heads, C] (dtype), out: bf16 [rows, heads, C].  Row r sits at position
+ * pos[r] (device int32 [rows]); pos == NULL means position r % pos_mod.
+ * Pairs (2i, 2i+1) of the last rope_dims channels turn by pos * theta^(-2i/rope_dims).
+ */
+CSA_API csa_status csa_norm_rope(const void* x, csa_dtype dtype, int64_t rows, int heads, int C,
+                         const int32_t* pos, int64_t pos_mod, int norm, float eps, int rope_dims,
+                         float rope_theta, void* out, cudaStream_t stream);
+
+/*
+ * csa_quantize_mxfp4 -- MXFP4 encoding (dev.to "How DeepSeek-V4 Achieves ...": the
+ * lightning indexer runs in FP4), per 32-element block of each row:
+ *   E = smallest integer with amax <= 6 * 2^E, clamped to [-127, 127] (amax = 0 -> -127);
+ *   code = round-half-even(x / 2^E) onto the E2M1 grid {0,.5,1,1.5,2,3,4,6}, sign = sign of x;
+ *   scales[r, b] = E + 127; packed[r, i] holds element 2i (low nibble) and 2i+1 (high nibble).
+ * x: [rows, cols] (dtype); cols % 32 == 0; packed [rows, cols/2]; scales [rows, cols/32].
+ * Bit-exact: the encoding is a pure function of the input bits.
+ */
+CSA_API csa_status csa_quantize_mxfp4(const void* x, csa_dtype dtype, int64_t rows, int cols, uint8_t* packed,
+                              uint8_t* scales, cudaStream_t stream);
+
+/*
+ * csa_index_topk -- lightning indexer and top-k selector ("DeepSeek-V4: Million-Token
+ * Context", CSA stage: a small attention head scores every compressed block against
+ * the query and the top-k selector keeps the best; "Follow the white rabbit", indexer
+ * paragraph: low-precision first pass, top 1,024 at maximum context).
+ *
+ * For query n (sequence q_seq[n], position q_pos[n]) and every visible entry
+ * j < n_vis = min(n_entries[q_seq[n]], floor((q_pos[n]+1)/m)):
+ *   d[h]  = <deq(q[n,h,:]), deq(k[q_seq[n], j, :])>            (exact in float32)
+ *   S[j]  = float32 chain over h = 0..Hi-1: acc = fmaf(w[n,h], max(d[h], 0), acc), acc0 = 0
+ * idx_out[n, :] = the k entries with the largest S (ties -> lowest j), ascending,
+ * -1 padded; cnt_out[n] = min(k, n_vis).  score_out (optional, [Nq, E_max]) receives S
+ * for j < n_vis.
+ *
+ * q_fp4 [Nq, Hi, Di/2], q_scale [Nq, Hi, Di/32] (csa_quantize_mxfp4 layout); w float32
+ * [Nq, Hi]; q_pos, q_seq int32 [Nq]; k_fp4 [B, E_max, Di/2], k_scale [B, E_max, Di/32];
+ * n_entries int32 [B].  Supported: Hi in {4, 8, 16, 32, 64}, Di in {64, 128}, 1 <= k <= 2048.
+ * workspace: device scratch of csa_index_topk_workspace(Nq, E_max, k) bytes, 256-byte aligned.
+ */
+CSA_API csa_status csa_index_topk(int Nq, int Hi, int Di, int k, int m, const uint8_t* q_fp4,
+                          const uint8_t* q_scale, const float* w, const int32_t* q_pos,
+                          const int32_t* q_seq, int B, int E_max, const uint8_t* k_fp4,
+                          const uint8_t* k_scale, const int32_t* n_entries, int32_t* idx_out,
+                          int32_t* cnt_out, float* score_out, void* workspace, size_t ws_bytes,
+                          cudaStream_t stream);
+CSA_API size_t csa_index_topk_workspace(int Nq, int E_max, int k);
+
+/*
+ * csa_index_score / csa_topk_select -- the two halves of csa_index_topk, for callers
+ * that keep the score rows: csa_index_score writes S (definition above) into
+ * scores[n, j] (float32 [Nq, E_stride], E_stride >= E_max) for j < n_vis of query n and
+ * leaves the rest of the row untouched; csa_topk_select reads scores[n, 0:n_vis] and
+ * writes idx_out / cnt_out exactly as csa_index_topk does.  Same support limits.
+ */
+CSA_API csa_status csa_index_score(int Nq, int Hi, int Di, int m, const uint8_t* q_fp4, const uint8_t* q_scale,
+                                   const float* w, const int32_t* q_pos, const int32_t* q_seq, int B, int E_max,
+                                   const uint8_t* k_fp4, const uint8_t* k_scale, const int32_t* n_entries,
+                                   float* scores, int E_stride, cudaStream_t stream);
+CSA_API csa_status csa_topk_select(int Nq, int k, int m, const float* scores, int E_stride, const int32_t* q_pos,
+                                   const int32_t* q_seq, int B, int E_max, const int32_t* n_entries,
+                                   int32_t* idx_out, int32_t* cnt_out, cudaStream_t stream);
+
+/*
+ * csa_sparse_attn -- core shared-KV MQA of CSA ("DeepSeek-V4: Towards Highly Efficient
+ * ...", section 2.3: shared-KV multi-query attention over the k selected entries;
+ * "DeepSeek-V4: Million-Token Context": each query head attends to the picked set
+ * plus a sliding window of the very recent tokens).
+ *
+ * For query n at position t in sequence b, keys K_r (= values) are
+ *   entries[b, idx[n, r]] for r < cnt[n], then
+ *   window_kv[b, u - window_base[b]] for max(0, t-W+1, window_base[b]) <= u <= min(t, window_base[b]+Tw-1),
+ * and for each head h one softmax runs over all of them:
+ *   out[n,h] = sum_r softmax_r(scale * <q[n,h], K_r>) K_r,   lse[n,h] = log sum_r exp(scale * <q[n,h], K_r>).
+ * q bf16 [Nq, H, D] (already normalised and rotated); entries bf16 [B, E_max, D];
+ * idx int32 [Nq, k] (entries < 0 or >= E_max are skipped and flag CSA_DEVERR_INDEX);
+ * cnt int32 [Nq]; window_kv bf16 [B, Tw, D]; window_base int32 [B]; out bf16 [Nq, H, D];
+ * lse float32 [Nq, H] or NULL.  Supported: H == 64, D == 512, W <= 4096.
+ * workspace: csa_sparse_attn_workspace(Nq, H, D, k, W) bytes.
+ */
+CSA_API csa_status csa_sparse_attn(int Nq, int H, int D, int k, int W, float scale, const void* q,
+                           const int32_t* q_pos, const int32_t* q_seq, int B, int E_max,
+                           const void* entries, const int32_t* idx, const int32_t* cnt, int Tw,
+                           const void* window_kv, const int32_t* window_base, void* out, float* lse,
+                           void* workspace, size_t ws_bytes, cudaStream_t stream);
+CSA_API size_t csa_sparse_attn_workspace(int Nq, int H, int D, int k, int W);
+
+/*
+ * hca_attn -- HCA dense attention ("DeepSeek-V4: Million-Token Context", HCA stage:
+ * every query attends to all compressed entries, plain multi-query attention, plus a
+ * small sliding window of uncompressed tokens).  As csa_sparse_attn with the selected
+ * set replaced by every visible entry j < min(n_entries[b], floor((t+1)/mprime)).
+ * workspace: hca_attn_workspace(Nq, H, D, E_max, W) bytes.
+ */
+CSA_API csa_status hca_attn(int Nq, int H, int D, int mprime, int W, float scale, const void* q,
+                    const int32_t* q_pos, const int32_t* q_seq, int B, int E_max, const void* entries,
+                    const int32_t* n_entries, int Tw, const void* window_kv, const int32_t* window_base,
+                    void* out, float* lse, void* workspace, size_t ws_bytes, cudaStream_t stream);
+CSA_API size_t hca_attn_workspace(int Nq, int H, int D, int E_max, int W);
+
+/* Synchronises `stream`, returns the device error word of the current device in
+ * *code_out and clears it.  CSA_ERR_CUDA if the stream reports an error. */
+CSA_API csa_status csa_get_device_error(int32_t* code_out, cudaStream_t stream);
+
+/* Static description of a status code. */
+CSA_API const char* csa_status_string(csa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H */

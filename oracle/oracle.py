@@ -19,7 +19,7 @@ import numpy as np
 __all__ = [
     "build", "lib", "n_visible", "pool", "rmsnorm", "rope", "mxfp4_quantize", "mxfp4_dequantize",
     "index_scores", "topk", "attention", "hca_select", "csa_prefill", "hca_prefill", "csa_decode",
-    "window_rows", "prep_queries", "F64", "F32", "BF16",
+    "window_rows", "prep_queries", "entries_rows", "F64", "F32", "BF16",
 ]
 
 F64, F32, BF16 = 0, 1, 2
@@ -221,7 +221,8 @@ def prep_queries(q: np.ndarray, pos: np.ndarray, norm: bool, eps: float, rope_di
     return rope(x, np.asarray(pos, dtype=np.int64), rope_dims, theta)
 
 
-def _entries(kv, z, bias, m, overlap, norm, eps, rope_dims, theta):
+def entries_rows(kv, z, bias, m, overlap, norm, eps, rope_dims, theta):
+    """Compressed entries of one sequence: RoPE at m(j+1)-1 of RMSNorm (optional) of the pooled rows."""
     e = pool(kv, z, bias, m, overlap)
     if norm:
         e = rmsnorm(e, eps)
@@ -237,7 +238,7 @@ def csa_prefill(wl, inp: dict, b: int = 0, rows: np.ndarray | None = None):
     (default: all tokens)."""
     T = inp["kv"].shape[1]
     rows = np.arange(T) if rows is None else np.asarray(rows)
-    ent = _entries(inp["kv"][b], inp["z"][b], inp["bias"], wl.m, wl.overlap, wl.norm, wl.eps, wl.rope_dims,
+    ent = entries_rows(inp["kv"][b], inp["z"][b], inp["bias"], wl.m, wl.overlap, wl.norm, wl.eps, wl.rope_dims,
                    wl.theta)
     win = window_rows(inp["kv"][b], wl.norm, wl.eps, wl.rope_dims, wl.theta)
     qf = prep_queries(inp["q"][b][rows], rows, wl.norm, wl.eps, wl.rope_dims, wl.theta)
@@ -263,7 +264,7 @@ def hca_prefill(wl, inp: dict, b: int = 0, rows: np.ndarray | None = None):
     """Whole HCA prefill layer (pool with m', dense attention over all visible entries + window)."""
     T = inp["kv"].shape[1]
     rows = np.arange(T) if rows is None else np.asarray(rows)
-    ent = _entries(inp["kv"][b], inp["z"][b], inp["bias"], wl.m, False, wl.norm, wl.eps, wl.rope_dims, wl.theta)
+    ent = entries_rows(inp["kv"][b], inp["z"][b], inp["bias"], wl.m, False, wl.norm, wl.eps, wl.rope_dims, wl.theta)
     win = window_rows(inp["kv"][b], wl.norm, wl.eps, wl.rope_dims, wl.theta)
     qf = prep_queries(inp["q"][b][rows], rows, wl.norm, wl.eps, wl.rope_dims, wl.theta)
     q_seq = np.zeros(len(rows), dtype=np.int32)

@@ -1,0 +1,77 @@
+"""The C-ABI library builds, loads without a GPU and exports every declared entry point;
+host-side validation answers with status codes before any device work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from compressed_sparse_long_02_b200 import build as bld
+    bld.build()
+    from compressed_sparse_long_02_b200 import binding
+    return binding.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^CSA_API\s+[\w\s\*]+?\b(\w+)\(", text, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for fn in ("csa_compress", "csa_index_topk", "csa_sparse_attn", "hca_attn", "csa_quantize_mxfp4",
+               "csa_norm_rope", "csa_get_device_error", "csa_status_string"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for fn in declared_functions():
+        assert hasattr(L, fn), f"{fn} declared in csa.h but not exported"
+
+
+def test_status_strings(L):
+    L.csa_status_string.restype = ctypes.c_char_p
+    assert L.csa_status_string(0) == b"ok"
+    assert b"workspace" in L.csa_status_string(4)
+    assert L.csa_status_string(99) == b"unknown status"
+
+
+def test_validation_without_device(L):
+    from compressed_sparse_long_02_b200 import binding as B
+    P = ctypes.c_void_p
+    # null configuration
+    assert L.csa_compress(None, 1, 8, P(16), P(16), P(16), None, 2, None, None, None, None) == 1
+    cfg = B._PoolCfg(4, 1, 96, 0, 1e-6, 0, 1e4, 0)  # C = 96 is not supported
+    assert L.csa_compress(ctypes.byref(cfg), 1, 8, P(16), P(16), P(16), None, 2, None, None, None, None) == 3
+    cfg = B._PoolCfg(4, 1, 128, 0, 1e-6, 3, 1e4, 0)  # odd rope dims
+    assert L.csa_compress(ctypes.byref(cfg), 1, 8, P(16), P(16), P(16), None, 2, None, None, None, None) == 1
+    cfg = B._PoolCfg(4, 1, 128, 0, 1e-6, 0, 1e4, 0)  # misaligned input pointer
+    assert L.csa_compress(ctypes.byref(cfg), 1, 8, P(17), P(16), P(16), None, 2, None, None, None, None) == 2
+    # quantiser: cols not a multiple of 32
+    assert L.csa_quantize_mxfp4(P(16), 0, 4, 48, P(16), P(16), None) == 1
+    # indexer: unsupported head dim, E_max not a multiple of 8, workspace too small
+    assert L.csa_index_topk(1, 4, 96, 8, 4, *([P(16)] * 5), 1, 64, *([P(16)] * 5), None, P(16), 1 << 30,
+                            None) == 3
+    assert L.csa_index_topk(1, 4, 64, 8, 4, *([P(16)] * 5), 1, 60, *([P(16)] * 5), None, P(16), 1 << 30,
+                            None) == 3
+    assert L.csa_index_topk(1, 4, 64, 8, 4, *([P(16)] * 5), 1, 64, *([P(16)] * 5), None, P(16), 16, None) == 4
+    # attention: only H = 64, D = 512
+    assert L.csa_sparse_attn(1, 32, 512, 8, 128, ctypes.c_float(0.04), *([P(16)] * 3), 1, 64, P(16), P(16), P(16),
+                             128, P(16), P(16), P(16), None, P(16), 1 << 30, None) == 3
+    assert L.hca_attn(1, 64, 512, 0, 128, ctypes.c_float(0.04), *([P(16)] * 3), 1, 64, P(16), P(16), 128, P(16),
+                      P(16), P(16), None, P(16), 1 << 30, None) == 1
+
+
+def test_workspace_sizes(L):
+    from compressed_sparse_long_02_b200 import binding as B
+    assert B.csa_index_topk_workspace(32, 32768, 1024) >= 32 * 32768 * 4
+    # one query per SM or more: no split, no partials
+    assert B.csa_sparse_attn_workspace(8192, 64, 512, 512, 128) <= 256
+    # decode: split partials of fp32 [splits, 64, 512] per query
+    assert B.csa_sparse_attn_workspace(32, 64, 512, 1024, 128) >= 32 * 2 * 64 * 512 * 4
