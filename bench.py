@@ -204,6 +204,20 @@ def decode_step(wl, cache, step, ws, ev=None):
         ev[4].record()
 
 
+def capture_step(fn):
+    """Capture `fn` (a sequence of C-ABI calls on the current stream) into a CUDA graph."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
 def bench_decode(args, dist, peaks):
     import torch
     from compressed_sparse_long_02_b200 import binding as B
@@ -212,12 +226,15 @@ def bench_decode(args, dist, peaks):
     dev = torch.device("cuda", dist.local_rank)
     R = args.replicas
     caches, steps, ws = setup_decode(wl, dev, R)
+    for i in range(R):  # eager pass: sets kernel attributes before capture
+        decode_step(wl, caches[i], steps[i], ws)
+    torch.cuda.synchronize()
+    graphs = [capture_step(lambda i=i: decode_step(wl, caches[i], steps[i], ws)) for i in range(R)]
     for i in range(args.warmup):
-        decode_step(wl, caches[i % R], steps[i % R], ws)
+        graphs[i % R].replay()
     torch.cuda.synchronize()
     assert B.csa_get_device_error() == 0, "device error during warm-up"
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(dist.local_rank)
     clocks.start()
@@ -225,7 +242,7 @@ def bench_decode(args, dist, peaks):
     torch.cuda.synchronize()
     start.record()
     for i in range(args.steps):
-        decode_step(wl, caches[i % R], steps[i % R], ws, evs[i])
+        graphs[i % R].replay()
     end.record()
     torch.cuda.synchronize()
     dist.barrier()
@@ -234,7 +251,14 @@ def bench_decode(args, dist, peaks):
     ms = dist.max(ms_local)
     assert B.csa_get_device_error() == 0, "device error in the timed region"
 
-    per = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in
+    # per-call device time: the same steps run eagerly behind a GPU sleep, so that the
+    # calls queue up and execute back to back between the events
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        torch.cuda._sleep(2_000_000)
+        decode_step(wl, caches[i % R], steps[i % R], ws, evs[i])
+    torch.cuda.synchronize()
+    per = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in
            enumerate(["quantize", "index_score", "topk_select", "attention"])}
     nb = decode_bytes_per_query(wl)
     queries_per_step = wl.B * dist.world
@@ -255,9 +279,10 @@ def bench_decode(args, dist, peaks):
         "per_call_us": {k: round(v * 1e3, 2) for k, v in per.items()},
         "clocks": clk,
         "gpu_launches": args.steps * 5,  # quantize, index score, top-k, attention, split merge
+        "graph": "one CUDA graph per input replica, replayed back to back",
     }
     res["e2e"] = bench_decode_e2e(args, wl, caches, steps, ws, dist)
-    del caches, steps, ws
+    del graphs, caches, steps, ws
     torch.cuda.empty_cache()
     return wl, res
 
@@ -468,7 +493,7 @@ def main():
                 "data": "synthetic (seeded; N(0,1) caches and queries, U(0,1) head weights)",
                 "config": decode_config(wl, args), "roofline": res["roofline"],
                 "step_roofline": res["step_roofline"], "per_call_us": res["per_call_us"], "e2e": res["e2e"],
-                "clocks": res["clocks"], "gpu_launches": res["gpu_launches"]}
+                "clocks": res["clocks"], "gpu_launches": res["gpu_launches"], "launch": res["graph"]}
         if not args.no_secondary:
             sec_steps = 5
             line["prefill"] = bench_prefill("csa_prefill_8k", sec_steps, 2, dist, peaks)
