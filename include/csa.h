@@ -167,6 +167,33 @@ CSA_API csa_status csa_index_topk(int Nq, int Hi, int Di, int k, int m, const ui
 CSA_API size_t csa_index_topk_workspace(int Nq, int E_max, int k);
 
 /*
+ * csa_index_topk_static -- csa_index_topk for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is a deployment variant of the same computation.
+ *
+ * Who needs it: code that runs the indexer where allocating is not allowed or not
+ * wise -- a plugin or custom operator inside a framework that owns every byte of device
+ * memory, a serving loop that must never call cudaMalloc (it can synchronise the whole
+ * device), a process whose memory a pool reserved up front.  The caller still provides
+ * every input and output; the only scratch, the float32 score rows, lives in a fixed
+ * 8 MiB device array inside this library, which every GPU that loads the library holds
+ * until the process exits.
+ *
+ * Arguments, results and support limits are those of csa_index_topk, without the
+ * workspace.  Size limit: Nq * round_up(E_max, 4) <= 2^21 scores (e.g. 32 queries of
+ * 65536 entries); larger calls return CSA_ERR_WORKSPACE and do nothing.
+ * The first call on a device looks up the array's device address with that device
+ * current; make that first call before any stream capture.  All calls share the one
+ * array: two calls that can run at the same time on the GPU (streams without an order
+ * between them) race on it.  No part of it has to start at zero: every score a call
+ * reads was written earlier by the same call.  Allocates nothing.
+ */
+CSA_API csa_status csa_index_topk_static(int Nq, int Hi, int Di, int k, int m, const uint8_t* q_fp4,
+                                         const uint8_t* q_scale, const float* w, const int32_t* q_pos,
+                                         const int32_t* q_seq, int B, int E_max, const uint8_t* k_fp4,
+                                         const uint8_t* k_scale, const int32_t* n_entries, int32_t* idx_out,
+                                         int32_t* cnt_out, cudaStream_t stream);
+
+/*
  * csa_index_score / csa_topk_select -- the two halves of csa_index_topk, for callers
  * that keep the score rows: csa_index_score writes S (definition above) into
  * scores[n, j] (float32 [Nq, E_stride], E_stride >= E_max) for j < n_vis of query n and
