@@ -67,6 +67,7 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 // one CTA = `epc` consecutive entries of one sequence; thread = channel pair
 template <bool kBf16>
 __global__ void pool_kernel(PoolArgs a, int epc) {
+  griddep_enter();
   __shared__ float red[32];
   const int b = blockIdx.y;
   const int E = a.T / a.m;
@@ -143,6 +144,7 @@ __global__ void pool_kernel(PoolArgs a, int epc) {
 // one CTA = one row (all heads); one warp per head vector, EPL consecutive channels per lane
 template <bool kBf16, int EPL>
 __global__ void norm_rope_kernel(NormRopeArgs a) {
+  griddep_enter();
   extern __shared__ float2 cs[];  // [rope_dims/2] (cos, sin) for this row's position
   const int64_t row = blockIdx.x;
   const int C = a.C;
@@ -194,15 +196,16 @@ cudaError_t launch_norm_rope_t(const NormRopeArgs& a, cudaStream_t s) {
   const int warps = a.heads < 8 ? a.heads : 8;
   const dim3 grid(static_cast<unsigned>(a.rows)), block(32 * warps);
   const size_t smem = sizeof(float2) * (a.rope_dims / 2 > 0 ? a.rope_dims / 2 : 1);
+  cudaError_t e = cudaSuccess;
   switch (a.C / 32) {
-    case 2: norm_rope_kernel<kBf16, 2><<<grid, block, smem, s>>>(a); break;
-    case 4: norm_rope_kernel<kBf16, 4><<<grid, block, smem, s>>>(a); break;
-    case 8: norm_rope_kernel<kBf16, 8><<<grid, block, smem, s>>>(a); break;
-    case 16: norm_rope_kernel<kBf16, 16><<<grid, block, smem, s>>>(a); break;
-    case 32: norm_rope_kernel<kBf16, 32><<<grid, block, smem, s>>>(a); break;
+    case 2: e = launch_pdl(norm_rope_kernel<kBf16, 2>, grid, block, smem, s, a); break;
+    case 4: e = launch_pdl(norm_rope_kernel<kBf16, 4>, grid, block, smem, s, a); break;
+    case 8: e = launch_pdl(norm_rope_kernel<kBf16, 8>, grid, block, smem, s, a); break;
+    case 16: e = launch_pdl(norm_rope_kernel<kBf16, 16>, grid, block, smem, s, a); break;
+    case 32: e = launch_pdl(norm_rope_kernel<kBf16, 32>, grid, block, smem, s, a); break;
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace
@@ -217,11 +220,8 @@ cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s) {
   if (E == 0 || (a.entries == nullptr && a.fp4 == nullptr)) return cudaSuccess;
   const int epc = a.m >= 32 ? 1 : (a.m >= 8 ? 4 : 16);
   const dim3 grid((E + epc - 1) / epc, a.B), block(a.C / 2);
-  if (a.in_bf16)
-    pool_kernel<true><<<grid, block, 0, s>>>(a, epc);
-  else
-    pool_kernel<false><<<grid, block, 0, s>>>(a, epc);
-  return cudaGetLastError();
+  return a.in_bf16 ? launch_pdl(pool_kernel<true>, grid, block, 0, s, a, epc)
+                   : launch_pdl(pool_kernel<false>, grid, block, 0, s, a, epc);
 }
 
 }  // namespace csa

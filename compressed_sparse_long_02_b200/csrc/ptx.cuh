@@ -12,6 +12,22 @@
 
 #include "csa.h"
 
+// Phase timestamps for development builds: CSA_T(slot, event) stores %globaltimer into
+// g_csa_timing[64][64], which a timing harness defines before including the kernel
+// sources; ordinary builds compile it to nothing.
+#ifdef CSA_TIMING
+#define CSA_T(slot, ev)                                                          \
+  do {                                                                           \
+    unsigned long long t_;                                                       \
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                       \
+    if ((slot) >= 0 && (slot) < 64 && (ev) >= 0 && (ev) < 64) g_csa_timing[slot][ev] = t_; \
+  } while (0)
+#else
+#define CSA_T(slot, ev) \
+  do {                  \
+  } while (0)
+#endif
+
 namespace csa {
 
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
@@ -96,6 +112,11 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, bool 
                : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 // make generic-proxy writes to shared memory visible to the async proxy (TMA, tcgen05)
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -212,6 +233,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
 __host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, uint32_t a_sf_id, uint32_t b_sf_id) {
   return ((b_sf_id & 3u) << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
          (static_cast<uint32_t>(M >> 4) << 24) | ((a_sf_id & 3u) << 29);
+}
+
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel of this library waits for the grid it depends on before its first global
+// memory access, and lets its own dependents launch right away; the dependents then sit
+// in the same wait, so only the launch latency overlaps (no data is touched early).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void griddep_enter() {
+  griddep_wait();
+  griddep_trigger();
 }
 
 // ------------------------------------------------------------------ misc

@@ -13,6 +13,7 @@ namespace {
 template <bool kBf16>
 __global__ void quantize_mxfp4_kernel(const void* __restrict__ x, int64_t n_pairs, uint8_t* __restrict__ packed,
                                       uint8_t* __restrict__ scales) {
+  griddep_enter();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   // the loop trip count is uniform across each warp because n_pairs % 16 == 0 and the
   // grid covers whole warps
@@ -51,10 +52,9 @@ cudaError_t launch_quantize_mxfp4(const void* x, int in_bf16, int64_t rows, int 
   const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
   if (blocks > cap) blocks = cap;
   if (in_bf16)
-    quantize_mxfp4_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, s>>>(x, n_pairs, packed, scales);
+    return launch_pdl(quantize_mxfp4_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, s, x, n_pairs, packed, scales);
   else
-    quantize_mxfp4_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, s>>>(x, n_pairs, packed, scales);
-  return cudaGetLastError();
+    return launch_pdl(quantize_mxfp4_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, s, x, n_pairs, packed, scales);
 }
 
 }  // namespace csa
