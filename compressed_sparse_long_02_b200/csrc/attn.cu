@@ -153,7 +153,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
+  CSA_TB(0);
   griddep_enter();
+  CSA_TB(1);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + kOffQ;
@@ -227,6 +229,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
   const uint32_t tmem = *tmem_slot;
   const int tslot = blockIdx.x < 2 ? 4 + static_cast<int>(blockIdx.x) : -1;
   if (threadIdx.x == 0) CSA_T(tslot, 0);
+  CSA_TB(2);
 
   if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------ gather producers
@@ -500,6 +503,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) CSA_T(tslot, 3);
+  CSA_TB(3);
   if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

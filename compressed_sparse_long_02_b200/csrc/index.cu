@@ -1,33 +1,31 @@
-// index_topk.cu -- lightning indexer (block-scaled FP4 tcgen05 contraction) and
-// exact radix top-k.
+// index.cu -- lightning indexer: block-scaled FP4 tcgen05 contraction of the query's
+// indexer heads against every visible compressed key, reduced to one score per entry.
 //
 // Sources: "DeepSeek-V4: Million-Token Context", CSA stage (a small attention head
-// scores every compressed block against the query; the top-k selector keeps the
-// best); "Follow the white rabbit: DeepSeek V4's architecture in 3D", indexer
-// paragraph (low-precision first pass adapted from V3.2's sparse attention, top
-// 1,024 at maximum context); dev.to "How DeepSeek-V4 Achieves Million-Token
-// Contexts ...", CSA paragraph (indexer in FP4).
+// scores every compressed block against the query); "Follow the white rabbit: DeepSeek
+// V4's architecture in 3D", indexer paragraph (low-precision first pass adapted from
+// V3.2's sparse attention); dev.to "How DeepSeek-V4 Achieves Million-Token Contexts
+// ...", CSA paragraph (indexer in FP4).
 //
 // Score of entry j for query n:  d[h] = <q[n,h], k[j]> (MXFP4 x MXFP4, exact in
 // fp32), S = fp32 chain acc = fmaf(w[n,h], max(d[h],0), acc) over h = 0..Hi-1.
 //
 // index_score_kernel -- one CTA per (query, run of entry tiles).  Entries go on the
 // MMA M axis (128 per tile), the query's heads on N, the head dim on K:
-//   warp 0      TMA producer: 128 FP4 key rows (SWIZZLE_64B) + their scale bytes per stage
-//   warp 1      TMEM owner and MMA issuer: rearranges the stage's scale bytes into the
-//               tcgen05 scale-factor layout, tcgen05.cp's them to TMEM and issues
+//   warp 0      TMA producer: the run's key scale bytes once, then 128 FP4 key rows
+//               (SWIZZLE_64B) per stage
+//   warp 1      TMEM owner and MMA issuer: rearranges the scale bytes into the tcgen05
+//               scale-factor layout, tcgen05.cp's them to TMEM once, then issues
 //               kind::mxf4.block_scale MMAs into a double-buffered accumulator
-//   warps 2..5  epilogue: one thread per entry (TMEM lane), ReLU, head-weighted fp32
-//               chain, store of the score row
-// topk_kernel -- one CTA per query row: 12/10/10-bit MSB radix select of the k-th
-// largest score (order-preserving float->uint key), then an ordered compaction that
-// keeps every score above the threshold and the lowest-index ties.
+//   warps 2..9  epilogue, two groups of four warps taking alternate tiles: one thread
+//               per entry (TMEM lane), ReLU, head-weighted fp32 chain, store of the score
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <cstdio>
 
+#include "common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 #include "tmap.h"
@@ -56,19 +54,15 @@ struct IndexParams {
   int32_t* err;
 };
 
-__device__ __forceinline__ int visible_entries(int pos, int m, int n_entries) {
-  int v = (pos + 1) / m;
-  v = v < 0 ? 0 : v;
-  return v < n_entries ? v : n_entries;
-}
-
 // kHi: number of indexer heads fixed at compile time (the head chain is straight-line
 // code), or 0 to take it from p.Hi at run time.
 template <int kHi>
 __global__ void __launch_bounds__(kIdxThreads, 2)
     index_score_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ksf,
                        const __grid_constant__ CUtensorMap tm_q, IndexParams p) {
+  CSA_TB(0);
   griddep_enter();
+  CSA_TB(1);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -135,6 +129,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
   const uint32_t tmem = *tmem_slot;
   const int tslot = blockIdx.x < 2 ? static_cast<int>(blockIdx.x) : -1;
   if (threadIdx.x == 0) CSA_T(tslot, 0);
+  CSA_TB(2);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -280,263 +275,14 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) CSA_T(tslot, 1);
+  CSA_TB(3);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
 }
 
-// ---------------------------------------------------------------------- top-k
-struct TopkParams {
-  const float* scores;
-  int E_stride, k, m, cache_cap, B, E_max;
-  const int32_t* q_pos;
-  const int32_t* q_seq;
-  const int32_t* n_entries;
-  int32_t* idx;
-  int32_t* cnt;
-};
-
-// order-preserving map of a float to uint32 (+0 and -0 map to the same key)
-__device__ __forceinline__ uint32_t order_key(float f) {
-  const uint32_t u = (f == 0.f) ? 0u : __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ void warp_hist_add(uint32_t* hist, uint32_t bin, bool active) {
-  const uint32_t peers = __match_any_sync(0xffffffffu, active ? bin : 0xFFFFFFFFu);
-  if (active && (threadIdx.x & 31) == static_cast<uint32_t>(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
-}
-
-// block-wide exclusive scan of one value per thread; returns the exclusive prefix, total in *tot
-template <int THREADS>
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_buf, uint32_t* tot) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += t;
-  }
-  if (lane == 31) warp_buf[warp] = inc;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t wv = lane < THREADS / 32 ? warp_buf[lane] : 0u;
-    uint32_t wi = wv;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += t;
-    }
-    if (lane < THREADS / 32) warp_buf[lane] = wi - wv;
-    if (lane == 31) *tot = wi;
-  }
-  __syncthreads();
-  const uint32_t r = warp_buf[warp] + inc - v;
-  __syncthreads();
-  return r;
-}
-
-// Find bin b with  #(bins above b) < need <= #(bins >= b).  Bins are scanned from the top.
-template <int THREADS>
-__device__ void select_bin(const uint32_t* hist, int nbins, uint32_t need, uint32_t* s_bin, uint32_t* s_above,
-                           uint32_t* warp_buf, uint32_t* tot) {
-  const int per = nbins / THREADS;
-  const int hi = nbins - per * static_cast<int>(threadIdx.x);  // bins [hi-per, hi)
-  uint32_t local = 0;
-  for (int i = 1; i <= per; ++i) local += hist[hi - i];
-  const uint32_t pre = block_excl_scan<THREADS>(local, warp_buf, tot);
-  if (pre < need && need <= pre + local) {
-    uint32_t acc = pre;
-    for (int i = 1; i <= per; ++i) {
-      const uint32_t c = hist[hi - i];
-      if (acc + c >= need) {
-        *s_bin = static_cast<uint32_t>(hi - i);
-        *s_above = acc;
-        break;
-      }
-      acc += c;
-    }
-  }
-  __syncthreads();
-}
-
-// Exact selection of the `need`-th largest key among n keys: three MSB digit passes
-// (12, 10, 10 bits).  Returns the threshold key and the number of keys above it.
-template <int THREADS, typename KeyFn>
-__device__ void radix_select(KeyFn key_of, int n, uint32_t need, uint32_t* hist, uint32_t* warp_buf,
-                             uint32_t* s_tot, uint32_t* s_bin, uint32_t* s_above, uint32_t& thr_out,
-                             uint32_t& above_out) {
-  uint32_t prefix = 0, above = 0;
-  const int shifts[3] = {20, 10, 0};
-  const int widths[3] = {12, 10, 10};
-#pragma unroll 1
-  for (int d = 0; d < 3; ++d) {
-    const int nb = 1 << widths[d];
-    for (int i = threadIdx.x; i < nb; i += THREADS) hist[i] = 0;
-    __syncthreads();
-    const int hi_shift = shifts[d] + widths[d];
-    for (int base = 0; base < n; base += THREADS) {
-      const int j = base + threadIdx.x;
-      const bool in = j < n;
-      const uint32_t key = in ? key_of(j) : 0u;
-      const bool act = in && (d == 0 || (key >> hi_shift) == prefix);
-      warp_hist_add(hist, (key >> shifts[d]) & static_cast<uint32_t>(nb - 1), act);
-    }
-    __syncthreads();
-    select_bin<THREADS>(hist, nb, need - above, s_bin, s_above, warp_buf, s_tot);
-    prefix = (prefix << widths[d]) | *s_bin;
-    above += *s_above;
-    __syncthreads();
-  }
-  thr_out = prefix;
-  above_out = above;
-}
-
-// One CTA per query row.  The row is staged in shared memory with all loads in flight;
-// scores are binned linearly over [min, max] of the row (an order-preserving map that
-// spreads concentrated score distributions over 4096 bins), the bin holding the k-th
-// largest is resolved exactly by radix select over its members, and an ordered
-// compaction writes every score above the threshold plus the lowest-index ties.  If
-// the threshold bin holds more members than the candidate buffer, the radix select
-// runs over the whole row instead (same result, slower).
-template <int THREADS>
-__global__ void __launch_bounds__(THREADS) topk_kernel(TopkParams p) {
-  griddep_enter();
-  extern __shared__ __align__(16) uint32_t tsm[];
-  constexpr int kCandCap = 8192;
-  uint32_t* hist = tsm;                 // 4096 bins
-  uint32_t* cand = tsm + 4096;          // candidate keys
-  uint32_t* rowbits = cand + kCandCap;  // cached score bits (cache_cap)
-  __shared__ uint32_t warp_buf[32], s_tot, s_bin, s_above, s_ncand;
-  __shared__ float s_red[2][32];
-
-  const int row = blockIdx.x;
-  const int seq = p.q_seq[row];
-  const int nv = (seq < 0 || seq >= p.B) ? 0 : min(visible_entries(p.q_pos[row], p.m, p.n_entries[seq]), p.E_max);
-  int32_t* out = p.idx + static_cast<size_t>(row) * p.k;
-  if (nv <= p.k) {
-    for (int j = threadIdx.x; j < p.k; j += THREADS) out[j] = j < nv ? j : -1;
-    if (threadIdx.x == 0) p.cnt[row] = nv;
-    return;
-  }
-  const float* src = p.scores + static_cast<size_t>(row) * p.E_stride;
-  const bool cached = nv <= p.cache_cap;
-  const int tslot = (row < 2 && threadIdx.x == 0) ? 2 + row : -1;
-  CSA_T(tslot, 0);
-  if (cached) {
-    const int n4 = (reinterpret_cast<uintptr_t>(src) & 15u) == 0 ? nv / 4 : 0;
-    for (int c = threadIdx.x; c < n4; c += THREADS) cp_async_16(smem_u32(rowbits + 4 * c), src + 4 * c, true);
-    for (int j = 4 * n4 + threadIdx.x; j < nv; j += THREADS) rowbits[j] = __float_as_uint(__ldg(src + j));
-    cp_async_wait_all();
-    __syncthreads();
-  }
-  CSA_T(tslot, 1);
-  auto val = [&](int j) -> float { return cached ? __uint_as_float(rowbits[j]) : __ldg(src + j); };
-  auto key_at = [&](int j) -> uint32_t { return order_key(val(j)); };
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int kWarps = THREADS / 32;
-
-  // row range
-  float lo = INFINITY, hi = -INFINITY;
-  for (int j = threadIdx.x; j < nv; j += THREADS) {
-    const float x = val(j);
-    lo = fminf(lo, x);
-    hi = fmaxf(hi, x);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-  }
-  if (lane == 0) {
-    s_red[0][warp] = lo;
-    s_red[1][warp] = hi;
-  }
-  for (int i = threadIdx.x; i < 4096; i += THREADS) hist[i] = 0;
-  if (threadIdx.x == 0) s_ncand = 0;
-  __syncthreads();
-  lo = s_red[0][0];
-  hi = s_red[1][0];
-  for (int w = 1; w < kWarps; ++w) {
-    lo = fminf(lo, s_red[0][w]);
-    hi = fmaxf(hi, s_red[1][w]);
-  }
-  const float span = hi - lo;
-  const float inv = (span > 0.f && span < INFINITY) ? 4095.0f / span : 0.f;
-  auto bin_of = [&](float x) -> uint32_t {  // monotone non-decreasing in x
-    const float f = (x - lo) * inv;
-    const uint32_t b = f > 0.f ? static_cast<uint32_t>(f) : 0u;
-    return b > 4095u ? 4095u : b;
-  };
-
-  // linear-bin histogram and the bin holding the k-th largest score
-  CSA_T(tslot, 2);
-  for (int j = threadIdx.x; j < nv; j += THREADS) atomicAdd(&hist[bin_of(val(j))], 1u);
-  __syncthreads();
-  CSA_T(tslot, 3);
-  select_bin<THREADS>(hist, 4096, static_cast<uint32_t>(p.k), &s_bin, &s_above, warp_buf, &s_tot);
-  const uint32_t b1 = s_bin;
-  const uint32_t above1 = s_above;
-  CSA_T(tslot, 4);
-  // members of that bin (keys strictly above lie in higher bins, below in lower ones)
-  for (int j = threadIdx.x; j < nv; j += THREADS) {
-    const float x = val(j);
-    if (bin_of(x) == b1) {
-      const uint32_t slot = atomicAdd(&s_ncand, 1u);
-      if (slot < kCandCap) cand[slot] = order_key(x);
-    }
-  }
-  __syncthreads();
-  const int ncand = static_cast<int>(s_ncand);
-  CSA_T(tslot, 5);
-  if (tslot >= 0) CSA_T(tslot, 40 + (ncand > 8192 ? 1 : 0));
-  uint32_t thr, n_above;
-  if (ncand <= kCandCap) {
-    uint32_t above_c;
-    radix_select<THREADS>([&](int i) { return cand[i]; }, ncand, static_cast<uint32_t>(p.k) - above1, hist, warp_buf,
-                          &s_tot, &s_bin, &s_above, thr, above_c);
-    n_above = above1 + above_c;
-  } else {
-    radix_select<THREADS>(key_at, nv, static_cast<uint32_t>(p.k), hist, warp_buf, &s_tot, &s_bin, &s_above, thr,
-                          n_above);
-  }
-  const uint32_t ties = static_cast<uint32_t>(p.k) - n_above;  // lowest-index keys equal to thr to keep
-  CSA_T(tslot, 6);
-
-  // ordered output: each warp owns a contiguous chunk; lanes stride through it so that
-  // ballots preserve index order
-  const int chunk = ((nv + kWarps - 1) / kWarps + 31) & ~31;
-  const int c_lo = warp * chunk, c_hi = min(nv, c_lo + chunk);
-  uint32_t n_gt = 0, n_eq = 0;
-  for (int base = c_lo; base < c_hi; base += 32) {
-    const int j = base + lane;
-    const uint32_t key = j < c_hi ? key_at(j) : 0u;
-    n_gt += __popc(__ballot_sync(0xffffffffu, j < c_hi && key > thr));
-    n_eq += __popc(__ballot_sync(0xffffffffu, j < c_hi && key == thr));
-  }
-  const uint32_t gt_pre = block_excl_scan<THREADS>(lane == 0 ? n_gt : 0u, warp_buf, &s_tot);
-  const uint32_t eq_pre = block_excl_scan<THREADS>(lane == 0 ? n_eq : 0u, warp_buf, &s_tot);
-  uint32_t gt_base = __shfl_sync(0xffffffffu, gt_pre, 0);
-  uint32_t eq_base = __shfl_sync(0xffffffffu, eq_pre, 0);
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int base = c_lo; base < c_hi; base += 32) {
-    const int j = base + lane;
-    const uint32_t key = j < c_hi ? key_at(j) : 0u;
-    const uint32_t bgt = __ballot_sync(0xffffffffu, j < c_hi && key > thr);
-    const uint32_t beq = __ballot_sync(0xffffffffu, j < c_hi && key == thr);
-    const uint32_t eq_before = eq_base + __popc(beq & lt_mask);
-    const bool take = (bgt >> lane & 1u) || ((beq >> lane & 1u) && eq_before < ties);
-    if (take) out[gt_base + __popc(bgt & lt_mask) + min(eq_before, ties)] = j;
-    gt_base += __popc(bgt);
-    eq_base += __popc(beq);
-  }
-  if (threadIdx.x == 0) p.cnt[row] = p.k;
-  CSA_T(tslot, 7);
-}
-
 int g_index_smem[2][64];
-int g_topk_smem[2][64];
 
 }  // namespace
 
@@ -590,38 +336,6 @@ cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s) {
   cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(index_score_kernel<0>), smem, g_index_smem[1]);
   if (e != cudaSuccess) return e;
   return launch_pdl(index_score_kernel<0>, dim3(a.Nq * p.splits), dim3(kIdxThreads), smem, s, tm_k, tm_ksf, tm_q, p);
-}
-
-cudaError_t launch_topk_select(const IndexArgs& a, cudaStream_t s) {
-  cudaError_t e = cudaSuccess;
-  TopkParams t{};
-  t.scores = a.scores_ws;
-  t.E_stride = a.E_stride;
-  t.k = a.k;
-  t.m = a.m;
-  t.B = a.B;
-  t.E_max = a.E_max;
-  t.q_pos = a.q_pos;
-  t.q_seq = a.q_seq;
-  t.n_entries = a.n_entries;
-  t.idx = a.idx_out;
-  t.cnt = a.cnt_out;
-  const bool big = a.E_max > 4096;
-  // dynamic limit leaves room for the kernel's static shared memory
-  const int max_dyn = 227 * 1024 - 1024;
-  const int cache_cap = std::min(a.E_max, (max_dyn - (4096 + 8192) * 4) / 4);
-  t.cache_cap = cache_cap;
-  const size_t tsmem = (4096 + 8192 + static_cast<size_t>(cache_cap)) * 4;
-  if (big) {
-    e = set_dyn_smem(reinterpret_cast<const void*>(topk_kernel<1024>), tsmem, g_topk_smem[1]);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(topk_kernel<1024>, dim3(a.Nq), dim3(1024), tsmem, s, t);
-  } else {
-    e = set_dyn_smem(reinterpret_cast<const void*>(topk_kernel<256>), tsmem, g_topk_smem[0]);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(topk_kernel<256>, dim3(a.Nq), dim3(256), tsmem, s, t);
-  }
-  return cudaGetLastError();
 }
 
 }  // namespace csa

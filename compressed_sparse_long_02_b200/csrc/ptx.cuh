@@ -22,9 +22,19 @@
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                       \
     if ((slot) >= 0 && (slot) < 64 && (ev) >= 0 && (ev) < 64) g_csa_timing[slot][ev] = t_; \
   } while (0)
+// CSA_TB(ev): per-CTA stamp into g_csa_cta[1024][4] (first 1024 CTAs), same builds only
+#define CSA_TB(ev)                                                               \
+  do {                                                                           \
+    unsigned long long t_;                                                       \
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                       \
+    if (threadIdx.x == 0 && blockIdx.x < 1024) g_csa_cta[blockIdx.x][ev] = t_;   \
+  } while (0)
 #else
 #define CSA_T(slot, ev) \
   do {                  \
+  } while (0)
+#define CSA_TB(ev) \
+  do {             \
   } while (0)
 #endif
 
