@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
             L.csa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
             L.csa_status_string.argtypes = [I]
             L.csa_status_string.restype = ctypes.c_char_p
+            L.csa_last_cuda_error.argtypes = []
+            L.csa_last_cuda_error.restype = ctypes.c_char_p
             for fn in ("csa_compress", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk", "csa_index_score",
                        "csa_topk_select", "csa_sparse_attn",
                        "hca_attn", "csa_get_device_error"):
@@ -76,7 +78,10 @@ def lib() -> ctypes.CDLL:
 
 def _check(fn: str, status: int):
     if status != 0:
-        raise CsaError(fn, status, lib().csa_status_string(status).decode())
+        msg = lib().csa_status_string(status).decode()
+        if status == 5:  # CSA_ERR_CUDA
+            msg += " (" + lib().csa_last_cuda_error().decode() + ")"
+        raise CsaError(fn, status, msg)
 
 
 def _ptr(t: torch.Tensor | None):

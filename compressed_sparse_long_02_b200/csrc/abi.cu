@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdio>
 #include <mutex>
 
 #include "csa.h"
@@ -21,9 +22,12 @@ std::mutex g_mu;
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool pow2_channels(int C) { return C == 64 || C == 128 || C == 256 || C == 512 || C == 1024; }
 
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
 csa_status from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return CSA_OK;
   if (e == cudaErrorInvalidValue) return CSA_ERR_INVALID_ARG;
+  g_last_cuda = e;
   return CSA_ERR_CUDA;
 }
 
@@ -58,6 +62,13 @@ int num_sms() {
 using namespace csa;
 
 extern "C" {
+
+const char* csa_last_cuda_error(void) {
+  thread_local char buf[256];
+  if (g_last_cuda == cudaSuccess) return "no error";
+  snprintf(buf, sizeof buf, "%s: %s", cudaGetErrorName(g_last_cuda), cudaGetErrorString(g_last_cuda));
+  return buf;
+}
 
 const char* csa_status_string(csa_status s) {
   switch (s) {

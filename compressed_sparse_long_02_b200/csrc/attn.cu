@@ -10,49 +10,68 @@
 // All H = 64 heads of one query share one key list, so a CTA works on one query
 // (or a contiguous split of its key list) and puts KEYS on the MMA M axis:
 //   S^T[128 keys, 64 heads]  = K[128 x 512] . Q^T           (K-major A and B, SW128)
-//   O^T[512 d, 64 heads]    += V^T[512 x 128] . P^T         (the same smem tile read
-//                                                            MN-major, P^T MN-major)
-// with K = V (shared KV).  S^T takes 64 TMEM columns, O^T 4 x 64.  Softmax runs one
-// thread per key (TMEM lane): head maxima and sums over keys are reduced with a
-// shuffle transpose-reduce (62 shuffles for 64 heads) and a 4-warp smem step.  The
-// running max is only moved when a tile raises it by more than 2^8, so O^T rarely
-// needs a rescale in TMEM.  Rows are gathered with cp.async (16-byte chunks, coalesced
-// 512-byte runs per warp) straight into the SWIZZLE_128B layout.
+//   O^T[512 d, 64 heads]    += V^T[512 x 128] . P^T         (V^T read MN-major, P^T MN-major)
+// with K = V (shared KV).
 //
-// Roles (288 threads): warps 0-3 softmax + epilogue, warps 4-7 gather producers,
-// warp 8 TMEM owner and MMA issuer.  When a query's keys are split over several CTAs
-// (decode), each CTA writes an unnormalised fp32 partial and (max, sum); a merge
-// kernel combines them.
+// Pipeline.  A tile's 128 rows are gathered slab by slab (a slab = 64 of the 512 dims
+// x 128 rows = 16 KB, SWIZZLE_128B) into a ring of kRing slabs, in the order the MMA
+// warp consumes them:  K0 | K1 V0 | K2 V1 | ... | V(n-1).  The K pass of a tile reads
+// its rows from HBM; the V pass gathers the same rows again (now in L2) once the
+// tile's probabilities exist, so the ring never has to hold a whole tile and QK of tile
+// i+1 runs while the softmax works on tile i.  S^T is double-buffered in TMEM (2 x 64
+// columns), P in shared memory (2 x 16 KB); O^T takes 4 x 64 TMEM columns.
+//
+// Softmax: one thread per (key row, 32 heads); the running max only moves when a tile
+// raises it by more than 2^8 (then O^T is rescaled in TMEM); sums over keys stay per
+// thread and are reduced once at the end.
+//
+// Roles (416 threads): warps 0-7 softmax + epilogue, warps 8-11 gather producers
+// (cp.async, 16-byte chunks; Q arrives by TMA), warp 12 TMEM owner and MMA issuer.  When a query's keys are split over several CTAs
+// (few queries), the splits of a query form a thread-block cluster: each CTA writes an
+// unnormalised fp32 partial and its (max, sum) to the workspace, the cluster
+// synchronises, and CTA r combines heads [r H/S, (r+1) H/S) of the query.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
 #include <cmath>
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "tmap.h"
 
 namespace csa {
 namespace {
 
 constexpr int kH = 64;
 constexpr int kD = 512;
-constexpr int kBN = 128;  // keys per tile
-constexpr int kAttnThreads = 416;  // 8 softmax warps, 4 gather warps, 1 MMA warp
+constexpr int kBN = 128;            // keys per tile
+constexpr int kSlabs = 8;           // 64-dim slabs per tile
+constexpr int kSlabBytes = 16384;
+constexpr int kRing = 6;            // even: the two slabs of a 128-dim PV chunk sit in adjacent slots
+constexpr int kProdWarps = 4;                          // gather producers
+constexpr int kRowsPerProd = (kBN + kProdWarps - 1) / kProdWarps;  // rows of a tile per producer warp
+static_assert(kRowsPerProd <= 32, "one row per lane");
+constexpr int kProdThreads = 32 * kProdWarps;
+constexpr int kMmaWarp = 8 + kProdWarps;               // TMEM owner and MMA issuer
+constexpr int kAttnThreads = 32 * (kMmaWarp + 1);      // 8 softmax warps first
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;
-constexpr uint32_t kColO = 64;
+constexpr uint32_t kColS = 0;       // 2 x 64 columns
+constexpr uint32_t kColO = 128;     // 4 x 64 columns
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kSplitSMs = 148;            // B200 SM count used to size decode splits
+constexpr int kSplitSMs = 148;             // B200 SM count used to size decode splits
+constexpr int kMaxSplits = 8;              // portable cluster size
 
-constexpr size_t kOffQ = 0;                      // 64 KB: [8 d-atoms][64 heads][128 B]
-constexpr size_t kOffKV = 64 * 1024;             // 128 KB: [8 d-atoms][128 keys][128 B]
-constexpr size_t kOffP = kOffKV + 128 * 1024;    // 16 KB: [128 keys][128 B]
-constexpr size_t kOffSmall = kOffP + 16 * 1024;  // reductions, running stats, barriers
-constexpr size_t kOffIdx = kOffSmall + 4096;     // 8 KB: this CTA's slice of the index list
+constexpr size_t kOffQ = 0;                                       // 64 KB: [8 d-atoms][64 heads][128 B]
+constexpr size_t kOffRing = 64 * 1024;                            // kRing x 16 KB
+constexpr size_t kOffP = kOffRing + kRing * kSlabBytes;           // 2 x 16 KB: [128 keys][128 B] x 8 atoms
+constexpr size_t kOffSmall = kOffP + 2 * 16384;                   // reductions, stats, barriers
+constexpr size_t kOffIdx = kOffSmall + 4096;                      // this CTA's slice of the index list
 constexpr int kIdxCap = 2048;
-constexpr size_t kAttnSmem = kOffIdx + 4 * kIdxCap + 1024;
-constexpr int kSlabLag = 3;  // cp.async groups (16 KB slabs) a producer keeps in flight
+constexpr size_t kAttnSmem = kOffIdx + 4 * kIdxCap + 1024;        // + alignment slack
+static_assert(kAttnSmem <= 227 * 1024, "shared memory budget");
+static_assert(kRing % 2 == 0, "ring shape");
 
 struct AttnParams {
   int Nq, k, W, B, E_max, Tw, mprime, dense;
@@ -74,6 +93,7 @@ struct AttnParams {
   int32_t* err;
 };
 
+// A query's key list: n_sel entries, then n_win window rows.
 struct KeyList {
   int b, n_sel, n_win;
   int64_t u_lo, wbase;
@@ -107,26 +127,6 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {  // byte offset 
   return static_cast<uint32_t>(row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
 }
 
-// 64 per-thread values (one per head) reduced over the 32 lanes of the warp; on
-// return v[0], v[1] hold the warp totals of heads 2*lane and 2*lane+1.
-template <bool kMax>
-__device__ __forceinline__ void xreduce64(float (&v)[64]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int lvl = 0; lvl < 5; ++lvl) {
-    const int off = 16 >> lvl;
-    const int half = 32 >> lvl;
-    const bool up = (lane & off) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float send = up ? v[i] : v[i + half];
-      const float keep = up ? v[i + half] : v[i];
-      const float got = __shfl_xor_sync(0xffffffffu, send, off);
-      v[i] = kMax ? fmaxf(keep, got) : keep + got;
-    }
-  }
-}
-
 // 32 per-thread values (one per head) reduced over the 32 lanes of the warp; on return
 // v[0] holds the warp total of head `lane`.
 template <bool kMax>
@@ -152,66 +152,77 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
-  CSA_TB(0);
-  griddep_enter();
-  CSA_TB(1);
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+// Stage st of the slab sequence K0 | K1 V0 | K2 V1 | ... | V(n-1): tile and pass.
+__device__ __forceinline__ void stage_of(int st, int n_tiles, int& tile, bool& is_v) {
+  if (st == 0) {
+    tile = 0;
+    is_v = false;
+  } else if (st == 2 * n_tiles - 1) {
+    tile = n_tiles - 1;
+    is_v = true;
+  } else if (st & 1) {
+    tile = (st + 1) >> 1;
+    is_v = false;
+  } else {
+    tile = (st >> 1) - 1;
+    is_v = true;
+  }
+}
+
+// every thread of every CTA in the cluster; release / acquire order global memory too
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// One CTA's share of a query: rows [row_begin, row_end) of its key list, n_tiles > 0.
+// Writes the normalised output (splits == 1) or the unnormalised partial + (max, sum).
+__device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& tm_q, uint8_t* smem, int n,
+                                       int split, const KeyList& kl,
+                                       int row_begin, int row_end, int n_tiles) {
   uint8_t* sQ = smem + kOffQ;
-  uint8_t* sKV = smem + kOffKV;
+  uint8_t* sRing = smem + kOffRing;
   uint8_t* sP = smem + kOffP;
   float* red_max = reinterpret_cast<float*>(smem + kOffSmall);  // [4][64]
   float* red_sum = red_max + 256;                                // [4][64]
   float* m_run = red_sum + 256;                                  // [64]
-  float* l_run = m_run + 64;                                // [64]
-  float* alpha = l_run + 64;                                // [64]
-  float* inv_l = alpha + 64;                                // [64]
-  uint8_t* row_ok = reinterpret_cast<uint8_t*>(inv_l + 64); // [128]: key row holds a valid source
-  uint64_t* bars = reinterpret_cast<uint64_t*>(row_ok + 128);
-  uint64_t* q_full = bars + 0;
-  uint64_t* slab_full = bars + 1;   // [8]: 16 KB slab (64 of the 512 dims) of the current tile loaded
-  uint64_t* slab_free = bars + 9;   // [8]: the MMAs reading that slab have completed
-  uint64_t* s_full = bars + 17;
-  uint64_t* p_full = bars + 18;
-  uint64_t* o_done = bars + 19;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
-  int32_t* sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);
+  float* l_run = m_run + 64;                                     // [64]
+  float* alpha = l_run + 64;                                     // [64]
+  float* inv_l = alpha + 64;                                     // [64]
+  uint8_t* row_ok = reinterpret_cast<uint8_t*>(inv_l + 64);      // [2][128]: key row has a valid source
+  uint64_t* bars = reinterpret_cast<uint64_t*>(row_ok + 256);
+  uint64_t* q_full = bars;                   // TMA: Q landed
+  uint64_t* full = q_full + 1;               // [kRing] producers: slab landed
+  uint64_t* slot_free = full + kRing;        // [kRing] MMA commit: slab consumed
+  uint64_t* s_full = slot_free + kRing;      // [2] MMA commit: S^T of a tile in TMEM
+  uint64_t* s_free = s_full + 2;             // [2] softmax warps: S^T read
+  uint64_t* p_full = s_free + 2;             // [2] softmax warps: P written (and O^T rescaled)
+  uint64_t* o_done = p_full + 2;             // MMA commit: PV of a tile complete
+  uint64_t* row_ready = o_done + 1;          // [2] producers: row_ok of a tile written
+  uint64_t* fin = row_ready + 2;             // MMA commit: every MMA of the CTA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int n = blockIdx.x / p.splits;
-  const int split = blockIdx.x % p.splits;
+  int32_t* sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (p.q_seq[n] < 0 || p.q_seq[n] >= p.B) {
-    if (threadIdx.x == 0) atomicExch(p.err, CSA_DEVERR_INDEX);
-    return;
-  }
-  const KeyList kl = key_list(p, n);
-  const int nk = kl.n_sel + kl.n_win;
-  const int row_begin = split * p.rows_per_split;
-  const int row_end = min(nk, row_begin + p.rows_per_split);
-  const int n_tiles = row_end > row_begin ? (row_end - row_begin + kBN - 1) / kBN : 0;
-
-  if (n_tiles == 0) {  // nothing to attend to in this split
-    if (p.splits == 1) {
-      for (int i = threadIdx.x; i < kH * kD / 2; i += blockDim.x)
-        reinterpret_cast<uint32_t*>(p.out + static_cast<size_t>(n) * kH * kD)[i] = 0u;
-      if (p.lse && threadIdx.x < kH) p.lse[n * kH + threadIdx.x] = -INFINITY;
-    } else if (threadIdx.x < kH) {
-      p.part_ml[(static_cast<size_t>(n) * p.splits + split) * kH + threadIdx.x] = make_float2(-INFINITY, 0.f);
-    }
-    return;
-  }
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 128);
-    for (int i = 0; i < 8; ++i) {
-      mbar_init(&slab_full[i], 128);
-      mbar_init(&slab_free[i], 1);
+    mbar_init(q_full, 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&full[i], kProdThreads);
+      mbar_init(&slot_free[i], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 8);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 8);
+      mbar_init(&p_full[b], 8);
+      mbar_init(&row_ready[b], kBN);
+    }
     mbar_init(o_done, 1);
+    mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -219,7 +230,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
     m_run[threadIdx.x] = -INFINITY;
     l_run[threadIdx.x] = 0.f;
   }
-  if (warp == 12) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -231,47 +242,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
   if (threadIdx.x == 0) CSA_T(tslot, 0);
   CSA_TB(2);
 
-  if (warp >= 8 && warp < 12) {
+  if (warp >= 8 && warp < 8 + kProdWarps) {
     // ------------------------------------------------------------ gather producers
+    // Producer warp pw owns rows [r0, r0 + nrows) of every tile; each lane resolves one of
+    // them and the warp issues their 8 x 16-byte chunks per slab.  The warps never wait on
+    // one another, so one that gives up cannot stall the others.
     const int pw = warp - 8;
     const int ptid = threadIdx.x - 256;
-    // this CTA's slice of the index list, staged once (no dependent global load per tile)
+    const int r0 = kRowsPerProd * pw;
+    const int nrows = min(kRowsPerProd, kBN - r0);
+    // this CTA's slice of the index list, staged once per warp (no dependent global load
+    // per row); each warp copies the part its own lanes will read
     const int sel_here = max(0, min(row_end, kl.n_sel) - row_begin);
     const bool staged = !p.dense && sel_here <= kIdxCap;
     if (staged)
-      for (int i = ptid; i < sel_here; i += 128) sidx[i] = p.idx[static_cast<size_t>(n) * p.k + row_begin + i];
-    named_bar_sync(2, 128);
-    {  // query: 64 head rows of 1 KB
-      const uint16_t* qb = p.q + static_cast<size_t>(n) * kH * kD;
-      for (int h = pw * 16; h < pw * 16 + 16; ++h) {
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int c = lane + 32 * half;
-          cp_async_16(smem_u32(sQ + (c >> 3) * 8192) + sw128(h, c), qb + h * kD + c * 8, true);
-        }
-      }
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(q_full);
-      if (ptid == 0) CSA_T(tslot, 1);
+      for (int i = lane; i < sel_here; i += 32)
+        if ((i % kBN) >= r0 && (i % kBN) < r0 + nrows)
+          sidx[i] = p.idx[static_cast<size_t>(n) * p.k + row_begin + i];
+    __syncwarp();
+    if (ptid == 0) {
+      prefetch_tmap(&tm_q);
+      // query: 64 head rows x 1 KB as 8 boxes of 64 rows x 128 B (one per 64-dim atom)
+      mbar_arrive_expect_tx(q_full, kH * kD * 2);
+      for (int a = 0; a < 8; ++a) tma_load_2d(smem_u32(sQ + a * 8192), &tm_q, q_full, 128 * a, n * kH);
     }
     bool ok = true;
-    for (int it = 0; ok && it < n_tiles; ++it) {
-      // slab 0 of the previous tile is free only after the softmax of that tile has
-      // arrived on p_full, i.e. after it read row_ok: row_ok may be rewritten now
-      if (it > 0 && !warp_wait(&slab_free[0], (it - 1) & 1, p.err, abort_flag)) break;
-      // each lane resolves the source of one of this warp's 32 rows
-      const int r_own = pw * 32 + lane;
-      const int g = row_begin + it * kBN + r_own;
+    int j = 0;  // slab sequence number
+    for (int st = 0; ok && st < 2 * n_tiles; ++st) {
+      int tile;
+      bool is_v;
+      stage_of(st, n_tiles, tile, is_v);
+      const int g = row_begin + tile * kBN + r0 + lane;
       const uint16_t* src = p.entries;
       bool valid = false;
-      if (g < row_end) {
+      if (lane < nrows && g < row_end) {
         if (g < kl.n_sel) {
           const int e = p.dense ? g : (staged ? sidx[g - row_begin] : p.idx[static_cast<size_t>(n) * p.k + g]);
           if (e >= 0 && e < p.E_max) {
             src = p.entries + (static_cast<size_t>(kl.b) * p.E_max + e) * kD;
             valid = true;
-          } else {
+          } else if (!is_v) {
             atomicExch(p.err, CSA_DEVERR_INDEX);
           }
         } else {
@@ -280,86 +290,120 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
           valid = true;
         }
       }
-      row_ok[r_own] = valid ? 1 : 0;  // read by the softmax after it observes slab_full[7]
       const unsigned long long src_ll = reinterpret_cast<unsigned long long>(src);
-      // slab by slab (64 dims x 128 rows = 16 KB): each instruction moves 4 rows x 128 B
-      for (int ka = 0; ka < 8; ++ka) {
-        if (it > 0 && ka > 0 && !warp_wait(&slab_free[ka], (it - 1) & 1, p.err, abort_flag)) {
+      for (int ka = 0; ka < kSlabs; ++ka, ++j) {
+        const int slot = j % kRing;
+        if (!warp_wait(&slot_free[slot], ((j / kRing) & 1) ^ 1, p.err, abort_flag)) {
           ok = false;
           break;
         }
-#pragma unroll
-        for (int rr = 0; rr < 32; rr += 4) {
-          const int rl = rr + (lane >> 3);
+        if (ptid == 0 && tslot == 4 && j < 64) CSA_T(10, j);
+        if (!is_v && ka == 0 && lane < nrows) {
+          // the softmax of the tile two back (same buffer) finished before this slot freed
+          row_ok[(tile & 1) * 128 + r0 + lane] = valid ? 1 : 0;
+          mbar_arrive(&row_ready[tile & 1]);
+          if (ptid == 0 && tile < 8) CSA_T(tslot, 8 + tile);
+        }
+        const uint32_t dst = smem_u32(sRing + slot * kSlabBytes);
+        for (int qb = 0; qb < 8 * nrows; qb += 32) {  // warp-uniform trip count: every lane shuffles
+          const int q = qb + lane;                      // chunk q: row r0 + q / 8, 16 bytes q % 8
+          const bool in = q < 8 * nrows;
+          const int rl = in ? q >> 3 : 0, c = q & 7;
           const uint16_t* rs = reinterpret_cast<const uint16_t*>(__shfl_sync(0xffffffffu, src_ll, rl));
           const bool rv = __shfl_sync(0xffffffffu, valid, rl);
-          const int c = lane & 7;
-          cp_async_16(smem_u32(sKV + ka * 16384) + sw128(pw * 32 + rl, c), rs + (ka * 8 + c) * 8, rv);
+          if (in) cp_async_16(dst + sw128(r0 + rl, c), rs + (ka * 8 + c) * 8, rv);
         }
-        cp_async_commit();
-        if (ka >= kSlabLag) {
-          cp_async_wait_group<kSlabLag>();
-          fence_proxy_async_smem();
-          mbar_arrive(&slab_full[ka - kSlabLag]);
-        }
+        // the slab's barrier completes when every producer thread's copies have landed;
+        // the consumer fences the async proxy after its wait
+        cp_async_mbar_arrive_noinc(&full[slot]);
       }
-      if (ptid == 0 && it < 8) CSA_T(tslot, 8 + it);
-      cp_async_wait_group<0>();
-      fence_proxy_async_smem();
-      if (ptid == 0 && it < 8) CSA_T(tslot, 16 + it);
-      if (ok)
-        for (int ka = 8 - kSlabLag; ka < 8; ++ka) mbar_arrive(&slab_full[ka]);
     }
-  } else if (warp == 12) {
+    cp_async_wait_all();  // nothing in flight when the CTA exits
+    {  // Q must have landed before the CTA may exit (already true on the normal path)
+      volatile int never = 0;
+      if (ptid == 0) mbar_wait(q_full, 0, p.err, &never);
+    }
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_qk = idesc_bf16(128, kH, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16(128, kH, true, true);
-    const uint32_t q0 = smem_u32(sQ), kv0 = smem_u32(sKV), p0 = smem_u32(sP);
+    const uint32_t q0 = smem_u32(sQ), ring0 = smem_u32(sRing), p0 = smem_u32(sP);
     bool ok = warp_wait(q_full, 0, p.err, abort_flag);
-    for (int it = 0; ok && it < n_tiles; ++it) {
-      // S^T = K Q^T, slab by slab as the slabs arrive
-      for (int ka = 0; ka < 8; ++ka) {
-        if (!warp_wait(&slab_full[ka], it & 1, p.err, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (lane == 0) {
+    int j = 0;
+    for (int st = 0; ok && st < 2 * n_tiles; ++st) {
+      int tile;
+      bool is_v;
+      stage_of(st, n_tiles, tile, is_v);
+      const int b = tile & 1;
+      if (!is_v) {
+        // S^T[b] = K Q^T slab by slab; buffer b was last read by the softmax of tile - 2
+        if (tile >= 2 && !warp_wait(&s_free[b], ((tile - 2) >> 1) & 1, p.err, abort_flag)) break;
+        for (int ka = 0; ka < kSlabs; ++ka, ++j) {
+          const int slot = j % kRing;
+          if (!warp_wait(&full[slot], (j / kRing) & 1, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0 && tslot == 4 && j < 64) CSA_T(12, j);
+          fence_proxy_async_smem();  // the producers' cp.async writes, seen through the barrier
+          tc_fence_after();
+          if (lane == 0) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + kColS, smem_desc(kv0 + ka * 16384 + kk * 32, 16, 1024, kSwizzle128B),
-                     smem_desc(q0 + ka * 8192 + kk * 32, 16, 1024, kSwizzle128B), idesc_qk, (ka | kk) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem + kColS + 64 * b,
+                       smem_desc(ring0 + slot * kSlabBytes + kk * 32, 16, 1024, kSwizzle128B),
+                       smem_desc(q0 + ka * 8192 + kk * 32, 16, 1024, kSwizzle128B), idesc_qk, (ka | kk) ? 1u : 0u);
+            tc_commit(&slot_free[slot]);
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          tc_commit(&s_full[b]);
+          if (tile < 8) CSA_T(tslot, 24 + tile);
+        }
+        __syncwarp();
+      } else {
+        // O^T += V^T P^T[b], one 128-dim chunk (two adjacent ring slots) at a time
+        if (!warp_wait(&p_full[b], (tile >> 1) & 1, p.err, abort_flag)) break;
+        tc_fence_after();
+        for (int dc = 0; dc < 4; ++dc, j += 2) {
+          const int slot = j % kRing;  // j even and kRing even: slot + 1 is the chunk's second slab
+          if (!warp_wait(&full[slot], (j / kRing) & 1, p.err, abort_flag) ||
+              !warp_wait(&full[slot + 1], ((j + 1) / kRing) & 1, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_smem();
+          tc_fence_after();
+          if (lane == 0) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              mma_bf16(tmem + kColO + 64 * dc,
+                       smem_desc(ring0 + slot * kSlabBytes + ks * 2048, kSlabBytes, 1024, kSwizzle128B),
+                       smem_desc(p0 + b * 16384 + ks * 2048, 16384, 1024, kSwizzle128B), idesc_pv,
+                       (tile > 0 || ks > 0) ? 1u : 0u);
+            tc_commit(&slot_free[slot]);
+            tc_commit(&slot_free[slot + 1]);
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          tc_commit(o_done);
+          if (tile < 8) CSA_T(tslot, 32 + tile);
         }
         __syncwarp();
       }
-      if (!ok) break;
-      if (lane == 0) tc_commit(s_full);
-      if (lane == 0 && it < 8) CSA_T(tslot, 24 + it);
-      __syncwarp();
-      if (!warp_wait(p_full, it & 1, p.err, abort_flag)) break;
-      tc_fence_after();
-      if (lane == 0) {
-        // O^T += V^T P^T; each 128-dim chunk frees its two slabs as soon as its MMAs retire
-#pragma unroll 1
-        for (int dc = 0; dc < 4; ++dc) {
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_bf16(tmem + kColO + 64 * dc, smem_desc(kv0 + 2 * dc * 16384 + ks * 2048, 16384, 1024, kSwizzle128B),
-                     smem_desc(p0 + ks * 2048, 16384, 1024, kSwizzle128B), idesc_pv, (it > 0 || ks > 0) ? 1u : 0u);
-          tc_commit(&slab_free[2 * dc]);
-          tc_commit(&slab_free[2 * dc + 1]);
-        }
-        tc_commit(o_done);
-        if (it < 8) CSA_T(tslot, 32 + it);
-      }
-      __syncwarp();
     }
+    // o_done may have two phases outstanding when the softmax finishes its last tile, so
+    // the epilogue waits on a barrier of its own
+    if (ok && lane == 0) tc_commit(fin);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax (warps 0-7)
     // thread = one key row of the tile (TMEM lane 32*(warp%4)+lane) and 32 heads
-    // (hh = warp/4 selects heads 0-31 or 32-63).  Sums over keys stay per thread in
-    // registers and are reduced once at the end; the running max is reduced only on the
-    // first tile or when a logit exceeds it by more than 2^8 (then O^T is rescaled).
+    // (hh = warp/4 selects heads 0-31 or 32-63).
     const int q4 = warp & 3, hh = warp >> 2;
     const int t = 32 * q4 + lane;
     const int h0 = 32 * hh;
@@ -367,38 +411,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
     float lacc[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) lacc[i] = 0.f;
+    bool ok = true;
     for (int it = 0; it < n_tiles; ++it) {
-      const bool got_s = mbar_wait(s_full, it & 1, p.err, abort_flag);
-      if (named_bar_or(1, 256, !got_s)) break;  // the group leaves together
+      const int b = it & 1;
+      const uint32_t ph = (it >> 1) & 1;
+      const bool got_s = mbar_wait(&s_full[b], ph, p.err, abort_flag);
+      if (named_bar_or(1, 256, !got_s)) {
+        ok = false;
+        break;
+      }
       if (t == 0 && hh == 0 && it < 8) CSA_T(tslot, 40 + it);
       tc_fence_after();
-      uint32_t sr[32];
-      tmem_ld16(tmem + lane_base + kColS + h0, sr);
-      tmem_ld16(tmem + lane_base + kColS + h0 + 16, sr + 16);
-      tmem_wait_ld();
-      // every producer wrote row_ok before arriving on slab_full[7] of this tile
-      const bool got_kv = mbar_wait(&slab_full[7], it & 1, p.err, abort_flag);
-      if (named_bar_or(1, 256, !got_kv)) break;
-      const bool valid = row_begin + it * kBN + t < row_end && row_ok[t] != 0;
+      const uint32_t s_addr = tmem + lane_base + kColS + 64 * b + h0;
+      const bool got_rows = mbar_wait(&row_ready[b], ph, p.err, abort_flag);
+      if (named_bar_or(1, 256, !got_rows)) {
+        ok = false;
+        break;
+      }
+      const bool valid = row_begin + it * kBN + t < row_end && row_ok[b * 128 + t] != 0;
+      // logits in log2 units; x is reused for the max reduction and the probabilities
       float x[32];
+      {
+        uint32_t sr[32];
+        tmem_ld16(s_addr, sr);
+        tmem_ld16(s_addr + 16, sr + 16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = valid ? __uint_as_float(sr[i]) * p.scale_log2 : -INFINITY;
+      }
       bool over = false;
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
         const float4 mm = *reinterpret_cast<const float4*>(m_run + h0 + i);
-        const float mv[4] = {mm.x, mm.y, mm.z, mm.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          x[i + j] = valid ? __uint_as_float(sr[i + j]) * p.scale_log2 : -INFINITY;
-          over |= x[i + j] > mv[j] + kRescaleThreshold;
-        }
+        over |= x[i] > mm.x + kRescaleThreshold;
+        over |= x[i + 1] > mm.y + kRescaleThreshold;
+        over |= x[i + 2] > mm.z + kRescaleThreshold;
+        over |= x[i + 3] > mm.w + kRescaleThreshold;
       }
-      const bool move_max = named_bar_or(1, 256, over);  // always true on the first tile
+      const bool move_max = named_bar_or(1, 256, over);  // always true on the first tile with a valid row
       if (move_max) {
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = x[i];
-        xreduce32<true>(v);
-        red_max[q4 * 64 + h0 + lane] = v[0];
+        xreduce32<true>(x);  // x[0] = this warp's max of head h0 + lane (x is reloaded below)
+        red_max[q4 * 64 + h0 + lane] = x[0];
         named_bar_sync(1, 256);
         if (threadIdx.x < kH) {
           const int h = threadIdx.x;
@@ -411,29 +464,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
         named_bar_sync(1, 256);
 #pragma unroll
         for (int i = 0; i < 32; ++i) lacc[i] *= alpha[h0 + i];
+        uint32_t sr[32];  // S^T[b] is intact until s_free[b] is arrived on below
+        tmem_ld16(s_addr, sr);
+        tmem_ld16(s_addr + 16, sr + 16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = valid ? __uint_as_float(sr[i]) * p.scale_log2 : -INFINITY;
       }
-      float pr[32];
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[b]);  // QK of tile it + 2 may overwrite S^T[b]
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
         const float4 mm = *reinterpret_cast<const float4*>(m_run + h0 + i);
-        pr[i] = valid ? exp2f(x[i] - mm.x) : 0.f;
-        pr[i + 1] = valid ? exp2f(x[i + 1] - mm.y) : 0.f;
-        pr[i + 2] = valid ? exp2f(x[i + 2] - mm.z) : 0.f;
-        pr[i + 3] = valid ? exp2f(x[i + 3] - mm.w) : 0.f;
+        x[i] = valid ? exp2f(x[i] - mm.x) : 0.f;
+        x[i + 1] = valid ? exp2f(x[i + 1] - mm.y) : 0.f;
+        x[i + 2] = valid ? exp2f(x[i + 2] - mm.z) : 0.f;
+        x[i + 3] = valid ? exp2f(x[i + 3] - mm.w) : 0.f;
       }
 #pragma unroll
-      for (int i = 0; i < 32; ++i) lacc[i] += pr[i];
-      // the P buffer and O^T are still in use by the previous tile's PV MMAs
-      const bool got_o = it == 0 || mbar_wait(o_done, (it - 1) & 1, p.err, abort_flag);
-      if (named_bar_or(1, 256, !got_o)) break;
-      tc_fence_after();
+      for (int i = 0; i < 32; ++i) lacc[i] += x[i];
+      float (&pr)[32] = x;
+      // P[b] was last read by PV of tile it - 2, which completed before QK of this tile
+      // signalled s_full (one thread issues both, and a commit covers every earlier MMA)
+      uint8_t* pb = sP + b * 16384;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const uint4 w4 = make_uint4(pack_bf16x2(pr[8 * c], pr[8 * c + 1]), pack_bf16x2(pr[8 * c + 2], pr[8 * c + 3]),
                                     pack_bf16x2(pr[8 * c + 4], pr[8 * c + 5]), pack_bf16x2(pr[8 * c + 6], pr[8 * c + 7]));
-        *reinterpret_cast<uint4*>(sP + sw128(t, 4 * hh + c)) = w4;
+        *reinterpret_cast<uint4*>(pb + sw128(t, 4 * hh + c)) = w4;
       }
-      if (move_max && it > 0) {  // move this warp's O^T columns (heads h0..h0+31) to the new max
+      if (move_max && it > 0) {
+        // move this warp's O^T columns (heads h0..h0+31) to the new max once PV of tile
+        // it - 1 is complete (PV of tile it waits for this warp's arrival on p_full)
+        const bool got_o = mbar_wait(o_done, (it - 1) & 1, p.err, abort_flag);
+        if (named_bar_or(1, 256, !got_o)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll 1
         for (int dc = 0; dc < 4; ++dc) {
           uint32_t o[32];
@@ -451,11 +520,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[b]);
       if (t == 0 && hh == 0 && it < 8) CSA_T(tslot, 48 + it);
     }
     // ------------------------------------------------------------ epilogue
-    const bool ok = !named_bar_or(1, 256, !mbar_wait(o_done, (n_tiles - 1) & 1, p.err, abort_flag));
+    const bool fin_ok = !named_bar_or(1, 256, !mbar_wait(fin, 0, p.err, abort_flag));  // all 256 take part
+    ok = ok && fin_ok;
     if (t == 0 && hh == 0) CSA_T(tslot, 2);
     tc_fence_after();
     xreduce32<false>(lacc);  // lane holds head h0+lane summed over this warp's 32 keys
@@ -484,19 +554,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
             ob[i * kD] = *reinterpret_cast<const uint16_t*>(&bv);
           }
         } else {
-          float* pb = p.part_o + ((static_cast<size_t>(n) * p.splits + split) * kH + h0) * kD + d;
+          float* pbo = p.part_o + ((static_cast<size_t>(n) * p.splits + split) * kH + h0) * kD + d;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) pb[i * kD] = __uint_as_float(o[i]);
+          for (int i = 0; i < 32; ++i) pbo[i * kD] = __uint_as_float(o[i]);
         }
       }
       if (threadIdx.x < kH) {
         const int h = threadIdx.x;
         if (p.splits == 1) {
-          if (p.lse) p.lse[n * kH + h] = (m_run[h] + log2f(l_run[h])) * 0.69314718055994531f;
+          if (p.lse) p.lse[n * kH + h] = l_run[h] > 0.f ? (m_run[h] + log2f(l_run[h])) * 0.69314718055994531f : -INFINITY;
         } else {
           p.part_ml[(static_cast<size_t>(n) * p.splits + split) * kH + h] = make_float2(m_run[h], l_run[h]);
         }
       }
+    } else if (threadIdx.x < kH && p.splits > 1) {  // gave up: this split contributes nothing
+      p.part_ml[(static_cast<size_t>(n) * p.splits + split) * kH + threadIdx.x] = make_float2(-INFINITY, 0.f);
     }
   }
 
@@ -504,58 +576,101 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnParams p) {
   __syncthreads();
   if (threadIdx.x == 0) CSA_T(tslot, 3);
   CSA_TB(3);
-  if (warp == 12) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
 }
 
-// one warp per (query, head): combine the split partials
-__global__ void attn_merge_kernel(const float* __restrict__ part_o, const float2* __restrict__ part_ml, int Nq,
-                                  int splits, uint16_t* __restrict__ out, float* __restrict__ lse) {
+__global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_constant__ CUtensorMap tm_q, AttnParams p) {
+  CSA_TB(0);
   griddep_enter();
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (gw >= Nq * kH) return;
-  const int n = gw / kH, h = gw % kH;
-  float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) {
-    const float2 ml = part_ml[(static_cast<size_t>(n) * splits + s) * kH + h];
-    if (ml.y > 0.f) M = fmaxf(M, ml.x);
+  CSA_TB(1);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int n = blockIdx.x / p.splits;
+  const int split = blockIdx.x % p.splits;  // the CTA's rank in its cluster when splits > 1
+  if (p.q_seq[n] < 0 || p.q_seq[n] >= p.B) {  // same for every CTA of the query (cluster)
+    if (threadIdx.x == 0 && split == 0) atomicExch(p.err, CSA_DEVERR_INDEX);
+    return;
   }
-  float L = 0.f;
-  float acc[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float2 ml = part_ml[(static_cast<size_t>(n) * splits + s) * kH + h];
-    if (!(ml.y > 0.f)) continue;
-    const float wgt = exp2f(ml.x - M);
-    L = fmaf(ml.y, wgt, L);
-    const float4* src =
-        reinterpret_cast<const float4*>(part_o + ((static_cast<size_t>(n) * splits + s) * kH + h) * kD) + lane * 4;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 v = __ldg(src + i);
-      acc[4 * i] = fmaf(v.x, wgt, acc[4 * i]);
-      acc[4 * i + 1] = fmaf(v.y, wgt, acc[4 * i + 1]);
-      acc[4 * i + 2] = fmaf(v.z, wgt, acc[4 * i + 2]);
-      acc[4 * i + 3] = fmaf(v.w, wgt, acc[4 * i + 3]);
+  const KeyList kl = key_list(p, n);
+  const int nk = kl.n_sel + kl.n_win;
+  const int row_begin = split * p.rows_per_split;
+  const int row_end = min(nk, row_begin + p.rows_per_split);
+  const int n_tiles = row_end > row_begin ? (row_end - row_begin + kBN - 1) / kBN : 0;
+
+  if (n_tiles > 0) {
+    attend(p, tm_q, smem, n, split, kl, row_begin, row_end, n_tiles);
+  } else if (p.splits == 1) {  // nothing to attend to
+    for (int i = threadIdx.x; i < kH * kD / 2; i += blockDim.x)
+      reinterpret_cast<uint32_t*>(p.out + static_cast<size_t>(n) * kH * kD)[i] = 0u;
+    if (p.lse && threadIdx.x < kH) p.lse[n * kH + threadIdx.x] = -INFINITY;
+  } else if (threadIdx.x < kH) {
+    p.part_ml[(static_cast<size_t>(n) * p.splits + split) * kH + threadIdx.x] = make_float2(-INFINITY, 0.f);
+  }
+  if (p.splits == 1) return;
+
+  // ---------------------------------------------------------------- combine the splits
+  // Every CTA of the cluster reaches this barrier (the branches above depend only on the
+  // query and the split), and the release / acquire pair orders the partials in global
+  // memory before the reads below.
+  __threadfence();
+  cluster_sync_all();
+  const int S = p.splits;
+  const int hp = kH / S;            // heads this CTA combines
+  const int hb = split * hp;
+  float* wsm = reinterpret_cast<float*>(smem);  // [hp][S] weights / L, then [hp] lse
+  if (static_cast<int>(threadIdx.x) < hp) {
+    const int h = hb + threadIdx.x;
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) {
+      const float2 ml = p.part_ml[(static_cast<size_t>(n) * S + s) * kH + h];
+      if (ml.y > 0.f) M = fmaxf(M, ml.x);
     }
+    float L = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float2 ml = p.part_ml[(static_cast<size_t>(n) * S + s) * kH + h];
+      const float w = ml.y > 0.f ? exp2f(ml.x - M) : 0.f;
+      wsm[threadIdx.x * S + s] = w;
+      L = fmaf(ml.y, w, L);
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    for (int s = 0; s < S; ++s) wsm[threadIdx.x * S + s] *= inv;
+    if (p.lse) p.lse[n * kH + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
   }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  uint32_t* o = reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(n) * kH + h) * kD + lane * 16);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) o[i] = pack_bf16x2(acc[2 * i] * inv, acc[2 * i + 1] * inv);
-  if (lse && lane == 0) lse[n * kH + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+  __syncthreads();
+  // hp heads x 512 dims, 4 dims per item
+  for (int it = threadIdx.x; it < hp * (kD / 4); it += blockDim.x) {
+    const int hl = it / (kD / 4), d4 = it % (kD / 4);
+    const int h = hb + hl;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < S; ++s) {
+      const float w = wsm[hl * S + s];
+      if (w == 0.f) continue;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                                  p.part_o + ((static_cast<size_t>(n) * S + s) * kH + h) * kD) + d4);
+      acc.x = fmaf(v.x, w, acc.x);
+      acc.y = fmaf(v.y, w, acc.y);
+      acc.z = fmaf(v.z, w, acc.z);
+      acc.w = fmaf(v.w, w, acc.w);
+    }
+    uint2 o2 = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+    *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(n) * kH + h) * kD + 4 * d4) = o2;
+  }
 }
 
 int g_attn_smem[64];
 
+// Splits of one query's key list: a power of two up to the portable cluster size, so
+// that the CTAs of a query fill about one wave of SMs.
 int split_count(int Nq, int max_keys) {
   const int tiles = std::max(1, (max_keys + kBN - 1) / kBN);
   if (Nq >= kSplitSMs) return 1;
-  return std::max(1, std::min(tiles, kSplitSMs / std::max(1, Nq)));
+  const int want = std::min(tiles, kSplitSMs / std::max(1, Nq));
+  int s = 1;
+  while (s * 2 <= want && s * 2 <= kMaxSplits) s *= 2;
+  return s;
 }
 
 }  // namespace
@@ -593,6 +708,10 @@ cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s) {
   const int splits = split_count(a.Nq, max_keys);
   p.splits = splits;
   p.rows_per_split = std::max(32, (((max_keys + splits - 1) / splits) + 31) / 32 * 32);
+  if (static_cast<int64_t>(a.Nq) * kH >= INT32_MAX) return cudaErrorInvalidValue;  // 32-bit TMA row coordinate
+  CUtensorMap tm_q;  // the queries as 64-row x 128-byte boxes
+  if (!encode_2d_u8(&tm_q, a.q, kD * 2, static_cast<uint64_t>(a.Nq) * kH, 128, kH, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   if (splits > 1) {
     const size_t o_bytes = static_cast<size_t>(a.Nq) * splits * kH * kD * sizeof(float);
     uintptr_t base = reinterpret_cast<uintptr_t>(a.ws);
@@ -602,11 +721,21 @@ cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s) {
   }
   cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(attn_kernel), kAttnSmem, g_attn_smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(attn_kernel, dim3(a.Nq * splits), dim3(kAttnThreads), kAttnSmem, s, p);
-  if (e != cudaSuccess || splits == 1) return e;
-  const int warps = a.Nq * kH;
-  return launch_pdl(attn_merge_kernel, dim3((warps * 32 + 255) / 256), dim3(256), 0, s,
-                    static_cast<const float*>(p.part_o), static_cast<const float2*>(p.part_ml), a.Nq, splits, a.out, a.lse);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.Nq * splits);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = kAttnSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(splits);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, attn_kernel, tm_q, p);
 }
 
 }  // namespace csa

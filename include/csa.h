@@ -252,6 +252,11 @@ CSA_API csa_status csa_get_device_error(int32_t* code_out, cudaStream_t stream);
 /* Static description of a status code. */
 CSA_API const char* csa_status_string(csa_status status);
 
+/* Name and description of the CUDA error behind the calling thread's most recent
+ * CSA_ERR_CUDA status (a static string; "no error" if there was none).  Calls that
+ * succeed do not clear it. */
+CSA_API const char* csa_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif
