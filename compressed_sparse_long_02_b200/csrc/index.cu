@@ -12,13 +12,15 @@
 //
 // index_score_kernel -- one CTA per (query, run of entry tiles).  Entries go on the
 // MMA M axis (128 per tile), the query's heads on N, the head dim on K:
-//   warp 0      TMA producer: the run's key scale bytes once, then 128 FP4 key rows
-//               (SWIZZLE_64B) per stage
-//   warp 1      TMEM owner and MMA issuer: rearranges the scale bytes into the tcgen05
-//               scale-factor layout, tcgen05.cp's them to TMEM once, then issues
-//               kind::mxf4.block_scale MMAs into a double-buffered accumulator
-//   warps 2..9  epilogue, two groups of four warps taking alternate tiles: one thread
-//               per entry (TMEM lane), ReLU, head-weighted fp32 chain, store of the score
+//   warp 0      TMA producer: key tile 0, the query, the run's key scale bytes (one bulk
+//               copy), then 128 FP4 key rows (SWIZZLE_64B) per stage
+//   warp 1      TMEM owner and MMA issuer: tcgen05.cp's the scale factors to TMEM once,
+//               then issues kind::mxf4.block_scale MMAs into a double-buffered accumulator
+//   warps 2..9  first rearrange the key scale bytes into the tcgen05 scale-factor layout
+//               (a tile per warp at a time), then the epilogue, two groups of four warps
+//               taking alternate tiles: one thread per entry (TMEM lane), ReLU,
+//               head-weighted fp32 chain, store of the score
+// Barrier set-up and the TMEM allocation run before the wait on the previous grid.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -33,7 +35,7 @@
 namespace csa {
 namespace {
 
-constexpr int kStages = 8;          // 8 KB key stages
+constexpr int kStages = 10;         // 8 KB key stages (two CTAs per SM)
 constexpr int kTileE = 128;
 constexpr int kMaxTilesPerCta = 31;  // all of a CTA's key scale factors stay in TMEM
 constexpr int kIdxThreads = 320;     // producer, MMA, two epilogue groups of four warps
@@ -49,6 +51,7 @@ struct IndexParams {
   const int32_t* q_seq;
   const int32_t* n_entries;
   const uint8_t* q_scale;
+  const uint8_t* k_scale;
   float* scores;
   float* score_out;
   int32_t* err;
@@ -58,53 +61,32 @@ struct IndexParams {
 // code), or 0 to take it from p.Hi at run time.
 template <int kHi>
 __global__ void __launch_bounds__(kIdxThreads, 2)
-    index_score_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ksf,
-                       const __grid_constant__ CUtensorMap tm_q, IndexParams p) {
+    index_score_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                       IndexParams p) {
   CSA_TB(0);
-  griddep_enter();
-  CSA_TB(1);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-  const int q = blockIdx.x / p.splits;
-  const int split = blockIdx.x % p.splits;
-  const int seq = p.q_seq[q];
-  if (seq < 0 || seq >= p.B) {  // bad sequence id: record it and produce nothing
-    if (threadIdx.x == 0 && split == 0) atomicExch(p.err, CSA_DEVERR_INDEX);
-    return;
-  }
-  const int nvis = min(visible_entries(p.q_pos[q], p.m, p.n_entries[seq]), p.E_max);
-  const int t_begin = split * p.tiles_per_cta;
-  const int t_end = min((nvis + kTileE - 1) / kTileE, t_begin + p.tiles_per_cta);
-  const int n_tiles = t_end - t_begin;
-  if (n_tiles <= 0) return;  // uniform: nothing allocated yet
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int Hi = kHi > 0 ? kHi : p.Hi;
-  const int row_bytes = p.Di / 2;            // 64 (Di=128) or 32 (Di=64)
-  const int a_bytes = kTileE * row_bytes;    // one stage of keys
-  const int sf_row = p.Di / 32;              // scale bytes per entry: 4 or 2
-  const int sf_bytes = kTileE * sf_row;      // 512 or 256
-  const int b_bytes = p.N * row_bytes;
-  const uint32_t swz = row_bytes == 64 ? kSwizzle64B : kSwizzle32B;
-  const uint32_t sbo = 8 * row_bytes;        // 8-row swizzle atom
 
   // shared memory carve-up
   uint8_t* sA = smem;                                    // kStages x 8 KB (1024-aligned)
   uint8_t* sB = sA + kStages * 8192;                     // 4 KB
-  uint8_t* sSF = sB + 4096;                              // kMaxTilesPerCta x 512: key scales, raw then atom
-  uint8_t* sSFB = sSF + kMaxTilesPerCta * 512;           // 512
+  uint8_t* sSF = sB + 4096;                              // kMaxTilesPerCta x 512: key scales, scale-factor layout
+  uint8_t* sSFraw = sSF + kMaxTilesPerCta * 512;         // kMaxTilesPerCta x 256: raw key scales when Di = 64
+  uint8_t* sSFB = sSFraw + kMaxTilesPerCta * 256;        // 512
   float* sW = reinterpret_cast<float*>(sSFB + 512);      // [64] head weights
   uint64_t* bars = reinterpret_cast<uint64_t*>(sW + 64);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
   uint64_t* b_full = bars + 2 * kStages;
-  uint64_t* sf_full = b_full + 1;
-  uint64_t* acc_full = sf_full + 1;
+  uint64_t* sf_full = b_full + 1;    // raw key scale bytes landed
+  uint64_t* sf_ready = sf_full + 1;  // epilogue warps: key scales rearranged
+  uint64_t* acc_full = sf_ready + 1;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  // Set-up that reads no global memory runs before the wait on the previous grid.
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -112,12 +94,15 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
     }
     mbar_init(b_full, 1);
     mbar_init(sf_full, 1);
+    mbar_init(sf_ready, 8);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);
     }
     *abort_flag = 0;
     fence_mbar_init();
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_q);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -127,34 +112,59 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_enter();
+  CSA_TB(1);
+
+  const int q = blockIdx.x / p.splits;
+  const int split = blockIdx.x % p.splits;
+  const int seq = p.q_seq[q];
+  const bool seq_ok = seq >= 0 && seq < p.B;
+  if (!seq_ok && threadIdx.x == 0 && split == 0) atomicExch(p.err, CSA_DEVERR_INDEX);  // produce nothing
+  const int nvis = seq_ok ? min(visible_entries(p.q_pos[q], p.m, p.n_entries[seq]), p.E_max) : 0;
+  const int t_begin = split * p.tiles_per_cta;
+  const int t_end = min((nvis + kTileE - 1) / kTileE, t_begin + p.tiles_per_cta);
+  const int n_tiles = t_end - t_begin;  // uniform over the CTA
+
+  const int Hi = kHi > 0 ? kHi : p.Hi;
+  const int row_bytes = p.Di / 2;            // 64 (Di=128) or 32 (Di=64)
+  const int a_bytes = kTileE * row_bytes;    // one stage of keys
+  const int sf_row = p.Di / 32;              // scale bytes per entry: 4 or 2
+  const int b_bytes = p.N * row_bytes;
+  const uint32_t swz = row_bytes == 64 ? kSwizzle64B : kSwizzle32B;
+  const uint32_t sbo = 8 * row_bytes;        // 8-row swizzle atom
   const int tslot = blockIdx.x < 2 ? static_cast<int>(blockIdx.x) : -1;
   if (threadIdx.x == 0) CSA_T(tslot, 0);
   CSA_TB(2);
 
-  if (warp == 0) {
+  if (n_tiles > 0 && warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_ksf);
-      prefetch_tmap(&tm_q);
-      // every key scale byte of this CTA's tiles, once (they stay in TMEM for the whole run)
-      mbar_arrive_expect_tx(sf_full, static_cast<uint32_t>(n_tiles * sf_bytes));
-      for (int i = 0; i < n_tiles; ++i)
-        tma_load_2d(smem_u32(sSF + i * 512), &tm_ksf, sf_full, 0,
-                    (seq * p.E_max + (t_begin + i) * kTileE) * sf_row / 16);
+      // key tile 0 first (the long pole), then the query, then every key scale byte of
+      // this CTA's tiles in one bulk copy (they stay in TMEM for the whole run), then the
+      // remaining key tiles as stages free up
+      const int row0 = seq * p.E_max + t_begin * kTileE;
+      mbar_arrive_expect_tx(&full[0], a_bytes);
+      CSA_T(tslot, 16);
+      tma_load_2d(smem_u32(sA), &tm_k, &full[0], 0, row0);
       mbar_arrive_expect_tx(b_full, b_bytes);
       tma_load_2d(smem_u32(sB), &tm_q, b_full, 0, q * Hi);
-      for (int it = 0; it < n_tiles; ++it) {
+      // entries with a scale byte in the cache: E_max and tile starts are multiples of 8,
+      // so the byte count is a multiple of 16
+      const int sf_entries = min(n_tiles * kTileE, p.E_max - t_begin * kTileE);
+      const uint32_t sf_bytes = static_cast<uint32_t>(sf_entries * sf_row);
+      mbar_arrive_expect_tx(sf_full, sf_bytes);
+      bulk_load(smem_u32(sf_row == 4 ? sSF : sSFraw), p.k_scale + static_cast<size_t>(row0) * sf_row, sf_bytes,
+                sf_full);
+      for (int it = 1; it < n_tiles; ++it) {
         const int st = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
         if (!mbar_wait(&empty[st], ph ^ 1, p.err, abort_flag)) break;
-        const int row = seq * p.E_max + (t_begin + it) * kTileE;
         mbar_arrive_expect_tx(&full[st], a_bytes);
         if (it < 16) CSA_T(tslot, 16 + it);
-        tma_load_2d(smem_u32(sA + st * 8192), &tm_k, &full[st], 0, row);
+        tma_load_2d(smem_u32(sA + st * 8192), &tm_k, &full[st], 0, row0 + it * kTileE);
       }
     }
-  } else if (warp == 1) {
+  } else if (n_tiles > 0 && warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // scale factors of B (the query's heads) into the tcgen05 scale-factor layout:
     // row r -> byte (r % 32) * 16 + (r / 32) * 4 + block; rows >= Hi are zero (2^-127)
@@ -176,41 +186,25 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
       if (lane == 0) tc_cp_32x128b_warpx4(tmem + kColSFB, smem_desc(smem_u32(sSFB), 0, 128, kSwizzleNone));
       __syncwarp();
     }
-    // key scale factors of all tiles: entry-major bytes -> scale-factor layout (in place per
-    // 512-byte slot), then one tcgen05.cp per tile into its own 4 TMEM columns
-    bool ok = warp_wait(sf_full, 0, p.err, abort_flag);
-    if (ok) {
-      for (int i = 0; i < n_tiles; ++i) {
-        uint8_t* slot = sSF + i * 512;
-        uint32_t words[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int r = lane + 32 * j;
-          words[j] = sf_row == 4 ? *reinterpret_cast<const uint32_t*>(slot + 4 * r)
-                                 : static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(slot + 2 * r));
-        }
-        __syncwarp();
-        *reinterpret_cast<uint4*>(slot + lane * 16) = make_uint4(words[0], words[1], words[2], words[3]);
-        __syncwarp();
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0)
-        for (int i = 0; i < n_tiles; ++i)
-          tc_cp_32x128b_warpx4(tmem + kColSFA + 4 * i, smem_desc(smem_u32(sSF + i * 512), 0, 128, kSwizzleNone));
-      __syncwarp();
-    }
-    ok = ok && warp_wait(b_full, 0, p.err, abort_flag);
-    for (int it = 0; ok && it < n_tiles; ++it) {
-      const int st = it % kStages;
-      const uint32_t ph = (it / kStages) & 1;
-      const int buf = it & 1;
-      if (!warp_wait(&full[st], ph, p.err, abort_flag)) break;
-      if (lane == 0 && it < 16) CSA_T(tslot, 32 + it);
-      if (!warp_wait(&acc_empty[buf], ((it >> 1) & 1) ^ 1, p.err, abort_flag)) break;
-      if (lane == 0 && it < 16 && tslot == 0) CSA_T(8, it);
-      tc_fence_after();
-      if (lane == 0) {
+    // key scale factors of every tile (rearranged by the epilogue warps): one tcgen05.cp
+    // per tile into its own 4 TMEM columns
+    bool ok = warp_wait(sf_ready, 0, p.err, abort_flag);
+    if (ok && lane == 0)
+      for (int i = 0; i < n_tiles; ++i)
+        tc_cp_32x128b_warpx4(tmem + kColSFA + 4 * i, smem_desc(smem_u32(sSF + i * 512), 0, 128, kSwizzleNone));
+    __syncwarp();
+    // one thread issues: no warp-wide polling or votes on the per-tile path
+    if (ok && lane == 0) {
+      ok = mbar_wait(b_full, 0, p.err, abort_flag);
+      for (int it = 0; ok && it < n_tiles; ++it) {
+        const int st = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        const int buf = it & 1;
+        if (!mbar_wait(&full[st], ph, p.err, abort_flag)) break;
+        if (it < 16) CSA_T(tslot, 32 + it);
+        if (!mbar_wait(&acc_empty[buf], ((it >> 1) & 1) ^ 1, p.err, abort_flag)) break;
+        if (it < 16 && tslot == 0) CSA_T(8, it);
+        tc_fence_after();
         const uint32_t sfa = tmem + kColSFA + 4 * it;
         const uint32_t a0 = smem_u32(sA + st * 8192), b0 = smem_u32(sB);
         for (int kh = 0; kh < p.Di / 64; ++kh) {
@@ -223,21 +217,40 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
         tc_commit(&acc_full[buf]);
         if (it < 16 && tslot == 0) CSA_T(9, it);
       }
-      __syncwarp();
     }
-  } else {
+    __syncwarp();
+  } else if (n_tiles > 0) {
     // ------------------------------------------------------------ epilogue (warps 2..9)
-    // group 0 (warps 2-5) takes even tiles / accumulator 0, group 1 (warps 6-9) odd tiles
-    // / accumulator 1, so two tiles are reduced at once
     const int ew = warp - 2;
-    const int grp = ew >> 2;
-    const int sub = warp & 3;  // TMEM lane quarter this warp may access
     if (ew * 32 + lane < 64) {
       const int h = ew * 32 + lane;
       sW[h] = h < Hi ? __ldg(p.w + static_cast<size_t>(q) * Hi + h) : 0.f;
     }
+    // key scales: entry-major bytes -> scale-factor layout, warp ew takes tiles ew, ew + 8, ...
+    // (word (r % 32) * 4 + r / 32 of a 512-byte slot holds the scale bytes of entry r)
+    bool ok = warp_wait(sf_full, 0, p.err, abort_flag);
+    if (ok) {
+      for (int i = ew; i < n_tiles; i += 8) {
+        uint32_t words[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = lane + 32 * j;
+          words[j] = sf_row == 4 ? *reinterpret_cast<const uint32_t*>(sSF + i * 512 + 4 * r)
+                                 : static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(sSFraw + i * 256 + 2 * r));
+        }
+        __syncwarp();
+        *reinterpret_cast<uint4*>(sSF + i * 512 + lane * 16) = make_uint4(words[0], words[1], words[2], words[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sf_ready);
+    }
     named_bar_sync(1, 256);
-    for (int it = grp; it < n_tiles; it += 2) {
+    // group 0 (warps 2-5) takes even tiles / accumulator 0, group 1 (warps 6-9) odd tiles
+    // / accumulator 1, so two tiles are reduced at once
+    const int grp = ew >> 2;
+    const int sub = warp & 3;  // TMEM lane quarter this warp may access
+    for (int it = grp; ok && it < n_tiles; it += 2) {
       const int buf = grp;
       if (!warp_wait(&acc_full[buf], (it >> 1) & 1, p.err, abort_flag)) break;
       if (sub == 0 && lane == 0 && it < 16 && tslot == 0) CSA_T(6, it);
@@ -294,12 +307,9 @@ size_t index_workspace_bytes(int Nq, int E_max, int /*k*/) {
 cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s) {
   const int row_bytes = a.Di / 2;
   const int N = std::max(16, (a.Hi + 15) / 16 * 16);
-  CUtensorMap tm_k, tm_ksf, tm_q;
+  CUtensorMap tm_k, tm_q;
   const CUtensorMapSwizzle swz = row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   if (!encode_2d_u8(&tm_k, a.k_fp4, row_bytes, static_cast<uint64_t>(a.B) * a.E_max, row_bytes, kTileE, swz))
-    return cudaErrorInvalidValue;
-  const uint64_t sf_total = static_cast<uint64_t>(a.B) * a.E_max * (a.Di / 32);
-  if (!encode_2d_u8(&tm_ksf, a.k_scale, 16, sf_total / 16, 16, kTileE * (a.Di / 32) / 16, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   if (!encode_2d_u8(&tm_q, a.q_fp4, row_bytes, static_cast<uint64_t>(a.Nq) * a.Hi, row_bytes, N, swz))
     return cudaErrorInvalidValue;
@@ -323,19 +333,20 @@ cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s) {
   p.q_seq = a.q_seq;
   p.n_entries = a.n_entries;
   p.q_scale = a.q_scale;
+  p.k_scale = a.k_scale;
   p.scores = a.scores_ws;
   p.score_out = a.score_out;
   p.err = device_error_word();
 
-  const size_t smem = 1024 + kStages * 8192 + 4096 + kMaxTilesPerCta * 512 + 512 + 256 + 512;
+  const size_t smem = 1024 + kStages * 8192 + 4096 + kMaxTilesPerCta * (512 + 256) + 512 + 256 + 512;
   if (a.Hi == 64) {
     cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(index_score_kernel<64>), smem, g_index_smem[0]);
     if (e != cudaSuccess) return e;
-    return launch_pdl(index_score_kernel<64>, dim3(a.Nq * p.splits), dim3(kIdxThreads), smem, s, tm_k, tm_ksf, tm_q, p);
+    return launch_pdl(index_score_kernel<64>, dim3(a.Nq * p.splits), dim3(kIdxThreads), smem, s, tm_k, tm_q, p);
   }
   cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(index_score_kernel<0>), smem, g_index_smem[1]);
   if (e != cudaSuccess) return e;
-  return launch_pdl(index_score_kernel<0>, dim3(a.Nq * p.splits), dim3(kIdxThreads), smem, s, tm_k, tm_ksf, tm_q, p);
+  return launch_pdl(index_score_kernel<0>, dim3(a.Nq * p.splits), dim3(kIdxThreads), smem, s, tm_k, tm_q, p);
 }
 
 }  // namespace csa
