@@ -266,30 +266,28 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
       mbar_arrive_expect_tx(q_full, kH * kD * 2);
       for (int a = 0; a < 8; ++a) tma_load_2d(smem_u32(sQ + a * 8192), &tm_q, q_full, 128 * a, n * kH);
     }
+    // source row of this lane in a tile (nullptr: no row; invalid indices are flagged once)
+    auto row_src = [&](int tile, bool flag) -> const uint16_t* {
+      const int g = row_begin + tile * kBN + r0 + lane;
+      if (lane >= nrows || g >= row_end) return nullptr;
+      if (g < kl.n_sel) {
+        const int e = p.dense ? g : (staged ? sidx[g - row_begin] : p.idx[static_cast<size_t>(n) * p.k + g]);
+        if (e >= 0 && e < p.E_max) return p.entries + (static_cast<size_t>(kl.b) * p.E_max + e) * kD;
+        if (flag) atomicExch(p.err, CSA_DEVERR_INDEX);
+        return nullptr;
+      }
+      const int64_t u = kl.u_lo + (g - kl.n_sel);
+      return p.window + (static_cast<size_t>(kl.b) * p.Tw + static_cast<size_t>(u - kl.wbase)) * kD;
+    };
     bool ok = true;
     int j = 0;  // slab sequence number
     for (int st = 0; ok && st < 2 * n_tiles; ++st) {
       int tile;
       bool is_v;
       stage_of(st, n_tiles, tile, is_v);
-      const int g = row_begin + tile * kBN + r0 + lane;
-      const uint16_t* src = p.entries;
-      bool valid = false;
-      if (lane < nrows && g < row_end) {
-        if (g < kl.n_sel) {
-          const int e = p.dense ? g : (staged ? sidx[g - row_begin] : p.idx[static_cast<size_t>(n) * p.k + g]);
-          if (e >= 0 && e < p.E_max) {
-            src = p.entries + (static_cast<size_t>(kl.b) * p.E_max + e) * kD;
-            valid = true;
-          } else if (!is_v) {
-            atomicExch(p.err, CSA_DEVERR_INDEX);
-          }
-        } else {
-          const int64_t u = kl.u_lo + (g - kl.n_sel);
-          src = p.window + (static_cast<size_t>(kl.b) * p.Tw + static_cast<size_t>(u - kl.wbase)) * kD;
-          valid = true;
-        }
-      }
+      const uint16_t* src_row = row_src(tile, !is_v);
+      const bool valid = src_row != nullptr;
+      const uint16_t* src = valid ? src_row : p.entries;
       const unsigned long long src_ll = reinterpret_cast<unsigned long long>(src);
       for (int ka = 0; ka < kSlabs; ++ka, ++j) {
         const int slot = j % kRing;

@@ -14,8 +14,9 @@
 // MMA M axis (128 per tile), the query's heads on N, the head dim on K:
 //   warp 0      TMA producer: key tile 0, the query, the run's key scale bytes (one bulk
 //               copy), then 128 FP4 key rows (SWIZZLE_64B) per stage
-//   warp 1      TMEM owner and MMA issuer: tcgen05.cp's the scale factors to TMEM once,
-//               then issues kind::mxf4.block_scale MMAs into a double-buffered accumulator
+//   warp 1      TMEM owner and MMA issuer: per tile, one thread tcgen05.cp's the tile's
+//               scale factors into a ring of TMEM slots and issues two
+//               kind::mxf4.block_scale MMAs into one of three accumulators
 //   warps 2..9  first rearrange the key scale bytes into the tcgen05 scale-factor layout
 //               (a tile per warp at a time), then the epilogue, two groups of four warps
 //               taking alternate tiles: one thread per entry (TMEM lane), ReLU,
@@ -37,11 +38,14 @@ namespace {
 
 constexpr int kStages = 10;         // 8 KB key stages (two CTAs per SM)
 constexpr int kTileE = 128;
-constexpr int kMaxTilesPerCta = 31;  // all of a CTA's key scale factors stay in TMEM
+constexpr int kMaxTilesPerCta = 31;  // a CTA stages all of its tiles' key scale bytes in shared memory
 constexpr int kIdxThreads = 320;     // producer, MMA, two epilogue groups of four warps
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColSFA = 128;    // 4 columns per tile: [128, 252)
-constexpr uint32_t kColSFB = 252;    // 4 columns
+constexpr int kAccBufs = 3;          // accumulators of 64 columns: [0, 192)
+constexpr int kSfRing = 8;           // key scale-factor slots of 4 columns: [192, 224)
+constexpr uint32_t kColSFA = 64 * kAccBufs;
+constexpr uint32_t kColSFB = kColSFA + 4 * kSfRing;  // 4 columns
+static_assert(kColSFB + 4 <= kTmemCols, "TMEM budget (two CTAs per SM)");
 
 struct IndexParams {
   int Nq, Hi, Di, m, B, E_max, E_stride, N;
@@ -82,8 +86,8 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
   uint64_t* sf_full = b_full + 1;    // raw key scale bytes landed
   uint64_t* sf_ready = sf_full + 1;  // epilogue warps: key scales rearranged
   uint64_t* acc_full = sf_ready + 1;
-  uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* acc_empty = acc_full + kAccBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + kAccBufs);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   // Set-up that reads no global memory runs before the wait on the previous grid.
@@ -95,7 +99,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
     mbar_init(b_full, 1);
     mbar_init(sf_full, 1);
     mbar_init(sf_ready, 8);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAccBufs; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);
     }
@@ -186,26 +190,24 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
       if (lane == 0) tc_cp_32x128b_warpx4(tmem + kColSFB, smem_desc(smem_u32(sSFB), 0, 128, kSwizzleNone));
       __syncwarp();
     }
-    // key scale factors of every tile (rearranged by the epilogue warps): one tcgen05.cp
-    // per tile into its own 4 TMEM columns
+    // key scale factors of every tile, rearranged by the epilogue warps; each tile's are
+    // copied into a ring of TMEM slots just before its MMAs (tcgen05 copies and MMAs of
+    // one thread run in issue order, so a slot is rewritten only after the MMAs reading it)
     bool ok = warp_wait(sf_ready, 0, p.err, abort_flag);
-    if (ok && lane == 0)
-      for (int i = 0; i < n_tiles; ++i)
-        tc_cp_32x128b_warpx4(tmem + kColSFA + 4 * i, smem_desc(smem_u32(sSF + i * 512), 0, 128, kSwizzleNone));
-    __syncwarp();
     // one thread issues: no warp-wide polling or votes on the per-tile path
     if (ok && lane == 0) {
       ok = mbar_wait(b_full, 0, p.err, abort_flag);
       for (int it = 0; ok && it < n_tiles; ++it) {
         const int st = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
-        const int buf = it & 1;
+        const int buf = it % kAccBufs;
         if (!mbar_wait(&full[st], ph, p.err, abort_flag)) break;
         if (it < 16) CSA_T(tslot, 32 + it);
-        if (!mbar_wait(&acc_empty[buf], ((it >> 1) & 1) ^ 1, p.err, abort_flag)) break;
+        if (!mbar_wait(&acc_empty[buf], ((it / kAccBufs) & 1) ^ 1, p.err, abort_flag)) break;
         if (it < 16 && tslot == 0) CSA_T(8, it);
         tc_fence_after();
-        const uint32_t sfa = tmem + kColSFA + 4 * it;
+        const uint32_t sfa = tmem + kColSFA + 4 * (it % kSfRing);
+        tc_cp_32x128b_warpx4(sfa, smem_desc(smem_u32(sSF + it * 512), 0, 128, kSwizzleNone));
         const uint32_t a0 = smem_u32(sA + st * 8192), b0 = smem_u32(sB);
         for (int kh = 0; kh < p.Di / 64; ++kh) {
           const uint32_t sf_id = 2 * kh;  // byte of the scale column holding blocks 2kh, 2kh+1
@@ -246,13 +248,13 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
       if (lane == 0) mbar_arrive(sf_ready);
     }
     named_bar_sync(1, 256);
-    // group 0 (warps 2-5) takes even tiles / accumulator 0, group 1 (warps 6-9) odd tiles
-    // / accumulator 1, so two tiles are reduced at once
+    // group 0 (warps 2-5) takes even tiles, group 1 (warps 6-9) odd tiles, so two tiles
+    // are reduced at once; tile it sits in accumulator it % kAccBufs
     const int grp = ew >> 2;
     const int sub = warp & 3;  // TMEM lane quarter this warp may access
     for (int it = grp; ok && it < n_tiles; it += 2) {
-      const int buf = grp;
-      if (!warp_wait(&acc_full[buf], (it >> 1) & 1, p.err, abort_flag)) break;
+      const int buf = it % kAccBufs;
+      if (!warp_wait(&acc_full[buf], (it / kAccBufs) & 1, p.err, abort_flag)) break;
       if (sub == 0 && lane == 0 && it < 16 && tslot == 0) CSA_T(6, it);
       tc_fence_after();
       uint32_t acc[64];

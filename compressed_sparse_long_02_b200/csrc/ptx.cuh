@@ -151,6 +151,10 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+// Hint: bring `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // Four rows (r0..r3) of a 2-D tensor, one box wide starting at column x, into 4 x box-width
 // bytes of shared memory at dst (128-byte aligned; the swizzle follows the address).
 // The tensor map's box must be one row high.  Rows past the end read as zeros.
