@@ -352,14 +352,27 @@ __global__ void __launch_bounds__(THREADS) topk_reg_kernel(TopkParams p) {
     s_zero = 0;
   }
 
+  // Per-slot passes come in two forms: a fully visible warp chunk (the common case, no
+  // per-slot validity test) and a partial one.
+  const bool full = valid == ~Mask(0);  // warp-uniform
+  auto slots = [&](auto body) {
+    if (full) {
+#pragma unroll
+      for (int i = 0; i < EPT; ++i) body(i, true);
+    } else {
+#pragma unroll
+      for (int i = 0; i < EPT; ++i) body(i, (valid >> i & kOne) != 0);
+    }
+  };
+
   // ---- range of the row
   float lo = INFINITY, hi = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < EPT; ++i)
-    if (valid >> i & kOne) {
+  slots([&](int i, bool ok) {
+    if (ok) {
       lo = fminf(lo, v[i]);
       hi = fmaxf(hi, v[i]);
     }
+  });
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
@@ -389,16 +402,19 @@ __global__ void __launch_bounds__(THREADS) topk_reg_kernel(TopkParams p) {
   const float span = hi - lo;
   const float inv = (span > 0.f && span < INFINITY) ? static_cast<float>(kBins - 1) / span : 0.f;
   const float nlo = inv > 0.f ? -lo * inv : 0.f;
-  // monotone non-decreasing in x (fma of an increasing affine map); NaN and negatives -> 0
+  // Bin of x: round(clamp(x inv - lo inv, 0, 4095)), monotone non-decreasing in x (an fma of
+  // an increasing affine map, then a clamp and a rounding); NaN -> 0.  Adding 1.5 * 2^23
+  // leaves the rounded integer in the low mantissa bits (no float-to-int conversion).
   auto bin_of = [&](float x, float c) -> uint32_t {
-    return min(__float2uint_rz(fmaf(x, inv, c)), static_cast<uint32_t>(kBins - 1));
+    const float f = fminf(fmaxf(fmaf(x, inv, c), 0.f), static_cast<float>(kBins - 1));
+    return __float_as_uint(f + 12582912.0f) - 0x4B400000u;
   };
   CSA_T(tslot, 1);
 
   // ---- histogram and the bin holding the k-th largest
-#pragma unroll
-  for (int i = 0; i < EPT; ++i)
-    if (valid >> i & kOne) atomicAdd(&hist[bin_of(v[i], nlo)], 1u);
+  slots([&](int i, bool ok) {
+    if (ok) atomicAdd(&hist[bin_of(v[i], nlo)], 1u);
+  });
   __syncthreads();
   select_bin<THREADS>(hist, kBins, static_cast<uint32_t>(p.k), &s_bin, &s_above, warp_buf, &s_tot);
   const uint32_t b1 = s_bin;
@@ -411,9 +427,9 @@ __global__ void __launch_bounds__(THREADS) topk_reg_kernel(TopkParams p) {
   Mask mem = 0;
   {
     const float c = nlo + __uint_as_float(*reinterpret_cast<volatile const uint32_t*>(&s_zero));
-#pragma unroll
-    for (int i = 0; i < EPT; ++i)
-      if ((valid >> i & kOne) && bin_of(v[i], c) == b1) mem |= kOne << i;
+    slots([&](int i, bool ok) {
+      if (ok && bin_of(v[i], c) == b1) mem |= kOne << i;
+    });
   }
 #pragma unroll
   for (int i = 0; i < EPT; ++i) {
@@ -484,16 +500,14 @@ __global__ void __launch_bounds__(THREADS) topk_reg_kernel(TopkParams p) {
   uint32_t mg[kHalves], me[kHalves];
 #pragma unroll
   for (int h = 0; h < kHalves; ++h) mg[h] = me[h] = 0;
-#pragma unroll
-  for (int i = 0; i < EPT; ++i) {
-    const bool ok = (valid >> i & kOne) != 0;
+  slots([&](int i, bool ok) {
     const uint32_t bg = __ballot_sync(0xffffffffu, ok && v[i] > thr_f);
     const uint32_t be = __ballot_sync(0xffffffffu, ok && v[i] == thr_f);
     if (lane == (i & 31)) {
       mg[i >> 5] = bg;
       me[i >> 5] = be;
     }
-  }
+  });
   // kept counts in order (half 0 lanes 0..31, then half 1), both <= 32768: 16-bit halves
   uint32_t incl[kHalves], cnt[kHalves];
   uint32_t wsum = 0;
