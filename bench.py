@@ -48,6 +48,33 @@ def load_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# ----------------------------------------------------------------------------- ncu traffic
+# DRAM bytes (read + write) per launch from one `ncu --set full` capture of the 128K
+# decode step (profiles/*_decode_128k.md), keyed by the sha1 of the kernel's source file
+# at capture time: a kernel changed since its capture reports traffic null.
+NCU_TRAFFIC = {
+    "attention": {"bytes": 40267520 + 761600, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
+                  "sha1": "67a07667369369326db30edc16e072746dca66f2"},
+    "index_score": {"bytes": 71479808 + 1585408, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
+                    "sha1": "0d868836e8e3b78c9d584e62b4bc2ac54fe9f374"},
+    "topk_select": {"bytes": 4260352, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",
+                    "sha1": "ef5746a9441cc408c3142e9e9c2489cef61a1b1e"},
+}
+
+
+def ncu_traffic(kernel: str):
+    import hashlib
+    e = NCU_TRAFFIC.get(kernel)
+    if e is None:
+        return None
+    try:
+        with open(os.path.join(ROOT, e["src"]), "rb") as f:
+            h = hashlib.sha1(f.read()).hexdigest()
+    except OSError:
+        return None
+    return e["bytes"] if h == e["sha1"] else None
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
@@ -272,7 +299,7 @@ def bench_decode(args, dist, peaks):
     res = {
         "value": value, "ms_per_step": ms_step,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": ncu_traffic(dom),
                      "algorithmic_bytes_per_launch": dom_bytes, "peak_source": peaks["source"]},
         "step_roofline": {"bound": "hbm", "algorithmic_bytes": nb["step"] * wl.B, "achieved_gbs": round(step_gbs, 1),
                           "frac": round(step_gbs / peaks["hbm_gbs"], 4)},
