@@ -179,65 +179,86 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   return r;
 }
 
+// Shared-memory layout of a CTA (one definition for the set-up and the pipeline).
+struct AttnSmem {
+  uint8_t* sQ;
+  uint8_t* sRing;
+  uint8_t* sP;
+  float* red_max;    // [4][64]
+  float* red_sum;    // [4][64]
+  float* m_run;      // [64]
+  float* l_run;      // [64]
+  float* alpha;      // [64]
+  float* inv_l;      // [64]
+  uint8_t* row_ok;   // [2][128]: key row has a valid source
+  uint64_t* q_full;     // TMA: Q landed
+  uint64_t* full;       // [kRing] producers: slab landed
+  uint64_t* slot_free;  // [kRing] MMA commit: slab consumed
+  uint64_t* s_full;     // [2] MMA commit: S^T of a tile in TMEM
+  uint64_t* s_free;     // [2] softmax warps: S^T read
+  uint64_t* p_full;     // [2] softmax warps: P written (and O^T rescaled)
+  uint64_t* o_done;     // MMA commit: PV of a tile complete
+  uint64_t* row_ready;  // [2] producers: row_ok of a tile written
+  uint64_t* fin;        // MMA commit: every MMA of the CTA complete
+  uint32_t* tmem_slot;
+  volatile int* abort_flag;
+  int32_t* sidx;        // this CTA's slice of the index list
+  __device__ explicit AttnSmem(uint8_t* smem) {
+    sQ = smem + kOffQ;
+    sRing = smem + kOffRing;
+    sP = smem + kOffP;
+    red_max = reinterpret_cast<float*>(smem + kOffSmall);
+    red_sum = red_max + 256;
+    m_run = red_sum + 256;
+    l_run = m_run + 64;
+    alpha = l_run + 64;
+    inv_l = alpha + 64;
+    row_ok = reinterpret_cast<uint8_t*>(inv_l + 64);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(row_ok + 256);
+    q_full = bars;
+    full = q_full + 1;
+    slot_free = full + kRing;
+    s_full = slot_free + kRing;
+    s_free = s_full + 2;
+    p_full = s_free + 2;
+    o_done = p_full + 2;
+    row_ready = o_done + 1;
+    fin = row_ready + 2;
+    tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+    abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);
+  }
+};
+
 // One CTA's share of a query: rows [row_begin, row_end) of its key list, n_tiles > 0.
 // Writes the normalised output (splits == 1) or the unnormalised partial + (max, sum).
-__device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& tm_q, uint8_t* smem, int n,
-                                       int split, const KeyList& kl,
-                                       int row_begin, int row_end, int n_tiles) {
-  uint8_t* sQ = smem + kOffQ;
-  uint8_t* sRing = smem + kOffRing;
-  uint8_t* sP = smem + kOffP;
-  float* red_max = reinterpret_cast<float*>(smem + kOffSmall);  // [4][64]
-  float* red_sum = red_max + 256;                                // [4][64]
-  float* m_run = red_sum + 256;                                  // [64]
-  float* l_run = m_run + 64;                                     // [64]
-  float* alpha = l_run + 64;                                     // [64]
-  float* inv_l = alpha + 64;                                     // [64]
-  uint8_t* row_ok = reinterpret_cast<uint8_t*>(inv_l + 64);      // [2][128]: key row has a valid source
-  uint64_t* bars = reinterpret_cast<uint64_t*>(row_ok + 256);
-  uint64_t* q_full = bars;                   // TMA: Q landed
-  uint64_t* full = q_full + 1;               // [kRing] producers: slab landed
-  uint64_t* slot_free = full + kRing;        // [kRing] MMA commit: slab consumed
-  uint64_t* s_full = slot_free + kRing;      // [2] MMA commit: S^T of a tile in TMEM
-  uint64_t* s_free = s_full + 2;             // [2] softmax warps: S^T read
-  uint64_t* p_full = s_free + 2;             // [2] softmax warps: P written (and O^T rescaled)
-  uint64_t* o_done = p_full + 2;             // MMA commit: PV of a tile complete
-  uint64_t* row_ready = o_done + 1;          // [2] producers: row_ok of a tile written
-  uint64_t* fin = row_ready + 2;             // MMA commit: every MMA of the CTA complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);
+__device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& tm_q, uint8_t* smem, uint32_t tmem,
+                                       int n, int split, const KeyList& kl, int row_begin, int row_end,
+                                       int n_tiles) {
+  const AttnSmem L(smem);
+  uint8_t* sQ = L.sQ;
+  uint8_t* sRing = L.sRing;
+  uint8_t* sP = L.sP;
+  float* red_max = L.red_max;
+  float* red_sum = L.red_sum;
+  float* m_run = L.m_run;
+  float* l_run = L.l_run;
+  float* alpha = L.alpha;
+  float* inv_l = L.inv_l;
+  uint8_t* row_ok = L.row_ok;
+  uint64_t* q_full = L.q_full;
+  uint64_t* full = L.full;
+  uint64_t* slot_free = L.slot_free;
+  uint64_t* s_full = L.s_full;
+  uint64_t* s_free = L.s_free;
+  uint64_t* p_full = L.p_full;
+  uint64_t* o_done = L.o_done;
+  uint64_t* row_ready = L.row_ready;
+  uint64_t* fin = L.fin;
+  volatile int* abort_flag = L.abort_flag;
+  int32_t* sidx = L.sidx;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int i = 0; i < kRing; ++i) {
-      mbar_init(&full[i], kProdThreads);
-      mbar_init(&slot_free[i], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 8);
-      mbar_init(&p_full[b], 8);
-      mbar_init(&row_ready[b], kBN);
-    }
-    mbar_init(o_done, 1);
-    mbar_init(fin, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (threadIdx.x < kH) {
-    m_run[threadIdx.x] = -INFINITY;
-    l_run[threadIdx.x] = 0.f;
-  }
-  if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
   const int tslot = blockIdx.x < 2 ? 4 + static_cast<int>(blockIdx.x) : -1;
   if (threadIdx.x == 0) CSA_T(tslot, 0);
   CSA_TB(2);
@@ -570,42 +591,97 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     }
   }
 
-  tc_fence_before();
-  __syncthreads();
   if (threadIdx.x == 0) CSA_T(tslot, 3);
   CSA_TB(3);
-  if (warp == kMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+}
+
+// Barriers, running statistics and the TMEM allocation: touches no global memory, so it
+// runs before the wait on the previous grid.  Returns the TMEM base address.
+__device__ __forceinline__ uint32_t attn_setup(uint8_t* smem) {
+  const AttnSmem L(smem);
+  float* m_run = L.m_run;
+  float* l_run = L.l_run;
+  uint64_t* q_full = L.q_full;
+  uint64_t* full = L.full;
+  uint64_t* slot_free = L.slot_free;
+  uint64_t* s_full = L.s_full;
+  uint64_t* s_free = L.s_free;
+  uint64_t* p_full = L.p_full;
+  uint64_t* o_done = L.o_done;
+  uint64_t* row_ready = L.row_ready;
+  uint64_t* fin = L.fin;
+  uint32_t* tmem_slot = L.tmem_slot;
+  volatile int* abort_flag = L.abort_flag;
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&full[i], kProdThreads);
+      mbar_init(&slot_free[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 8);
+      mbar_init(&p_full[b], 8);
+      mbar_init(&row_ready[b], kBN);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
+  if (threadIdx.x < kH) {
+    m_run[threadIdx.x] = -INFINITY;
+    l_run[threadIdx.x] = 0.f;
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return *tmem_slot;
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_constant__ CUtensorMap tm_q, AttnParams p) {
   CSA_TB(0);
-  griddep_enter();
-  CSA_TB(1);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (threadIdx.x == 0) prefetch_tmap(&tm_q);
+  const uint32_t tmem = attn_setup(smem);
+  griddep_enter();
+  CSA_TB(1);
   const int n = blockIdx.x / p.splits;
   const int split = blockIdx.x % p.splits;  // the CTA's rank in its cluster when splits > 1
-  if (p.q_seq[n] < 0 || p.q_seq[n] >= p.B) {  // same for every CTA of the query (cluster)
-    if (threadIdx.x == 0 && split == 0) atomicExch(p.err, CSA_DEVERR_INDEX);
-    return;
+  const bool seq_ok = p.q_seq[n] >= 0 && p.q_seq[n] < p.B;  // same for every CTA of the query (cluster)
+  if (!seq_ok && threadIdx.x == 0 && split == 0) atomicExch(p.err, CSA_DEVERR_INDEX);
+  KeyList kl{};
+  int row_begin = 0, row_end = 0, n_tiles = 0;
+  if (seq_ok) {
+    kl = key_list(p, n);
+    const int nk = kl.n_sel + kl.n_win;
+    row_begin = split * p.rows_per_split;
+    row_end = min(nk, row_begin + p.rows_per_split);
+    n_tiles = row_end > row_begin ? (row_end - row_begin + kBN - 1) / kBN : 0;
   }
-  const KeyList kl = key_list(p, n);
-  const int nk = kl.n_sel + kl.n_win;
-  const int row_begin = split * p.rows_per_split;
-  const int row_end = min(nk, row_begin + p.rows_per_split);
-  const int n_tiles = row_end > row_begin ? (row_end - row_begin + kBN - 1) / kBN : 0;
 
-  if (n_tiles > 0) {
-    attend(p, tm_q, smem, n, split, kl, row_begin, row_end, n_tiles);
-  } else if (p.splits == 1) {  // nothing to attend to
-    for (int i = threadIdx.x; i < kH * kD / 2; i += blockDim.x)
-      reinterpret_cast<uint32_t*>(p.out + static_cast<size_t>(n) * kH * kD)[i] = 0u;
-    if (p.lse && threadIdx.x < kH) p.lse[n * kH + threadIdx.x] = -INFINITY;
-  } else if (threadIdx.x < kH) {
-    p.part_ml[(static_cast<size_t>(n) * p.splits + split) * kH + threadIdx.x] = make_float2(-INFINITY, 0.f);
+  if (n_tiles > 0) attend(p, tm_q, smem, tmem, n, split, kl, row_begin, row_end, n_tiles);
+  tc_fence_before();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (!seq_ok) return;
+  if (n_tiles == 0) {  // nothing to attend to in this split
+    if (p.splits == 1) {
+      for (int i = threadIdx.x; i < kH * kD / 2; i += blockDim.x)
+        reinterpret_cast<uint32_t*>(p.out + static_cast<size_t>(n) * kH * kD)[i] = 0u;
+      if (p.lse && threadIdx.x < kH) p.lse[n * kH + threadIdx.x] = -INFINITY;
+    } else if (threadIdx.x < kH) {
+      p.part_ml[(static_cast<size_t>(n) * p.splits + split) * kH + threadIdx.x] = make_float2(-INFINITY, 0.f);
+    }
   }
   if (p.splits == 1) return;
 
