@@ -315,40 +315,65 @@ def bench_decode(args, dist, peaks):
 
 
 def bench_decode_e2e(args, wl, caches, steps, ws, dist):
-    """Decode through the public API with host buffers: pinned H2D of the step's inputs
-    (q, indexer query, head weights, positions) and D2H of the output, every step."""
+    """Decode through the public API with host buffers: every step copies its inputs (q,
+    indexer query, head weights, positions) from pinned host memory and its output back.
+    Steps are independent batches (the input replicas rotate), so they are pipelined
+    over three streams: the upload of step i+1 and the download of step i-1 overlap the
+    layer call of step i (two buffer sets, ordered by events)."""
     import torch
     from compressed_sparse_long_02_b200 import layer
     R = len(caches)
+    dev = ws["out"].device
     host = []
     for r in range(R):
         host.append({k: v.cpu().pin_memory() for k, v in steps[r].items()})
-    dev_in = {k: torch.empty_like(v) for k, v in steps[0].items()}
-    out_host = torch.empty((wl.B, wl.H, wl.D), dtype=torch.bfloat16).pin_memory()
+    NB = 2
+    dev_in = [{k: torch.empty_like(v) for k, v in steps[0].items()} for _ in range(NB)]
+    dev_out = [torch.empty((wl.B, wl.H, wl.D), dtype=torch.bfloat16, device=dev) for _ in range(NB)]
+    out_host = [torch.empty((wl.B, wl.H, wl.D), dtype=torch.bfloat16).pin_memory() for _ in range(NB)]
     h2d = sum(v.numel() * v.element_size() for v in host[0].values())
-    d2h = out_host.numel() * out_host.element_size()
+    d2h = out_host[0].numel() * out_host[0].element_size()
     lws = {"q_fp4": ws["q_fp4"], "q_scale": ws["q_scale"], "idx": ws["idx"], "cnt": ws["cnt"], "seq": ws["seq"],
            "attn_ws": ws["attn_ws"],
            "index_ws": torch.empty(layer.B.csa_index_topk_workspace(wl.B, wl.E, wl.k), dtype=torch.uint8,
-                                   device=ws["out"].device)}
+                                   device=dev)}
+    s_up, s_comp, s_down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_up = [torch.cuda.Event() for _ in range(NB)]
+    ev_comp = [torch.cuda.Event() for _ in range(NB)]
+    ev_down = [torch.cuda.Event() for _ in range(NB)]
 
-    def one(i):
-        src = host[i % R]
-        for k in dev_in:
-            dev_in[k].copy_(src[k], non_blocking=True)
-        r = layer.csa_decode(wl, caches[i % R], dev_in, lws, out=ws["out"])
-        out_host.copy_(r["out"], non_blocking=True)
-        torch.cuda.current_stream().synchronize()
+    def run(n0, n):
+        for i in range(n0, n0 + n):
+            b = i % NB
+            if i - n0 >= NB:
+                ev_down[b].synchronize()  # out_host[b] and dev_out[b] of step i - NB are free
+            with torch.cuda.stream(s_up):
+                s_up.wait_event(ev_comp[b])  # dev_in[b] no longer read by step i - NB
+                src = host[i % R]
+                for k in dev_in[b]:
+                    dev_in[b][k].copy_(src[k], non_blocking=True)
+                ev_up[b].record(s_up)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev_up[b])
+                s_comp.wait_event(ev_down[b])  # dev_out[b] downloaded
+                layer.csa_decode(wl, caches[i % R], dev_in[b], lws, out=dev_out[b])
+                ev_comp[b].record(s_comp)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(ev_comp[b])
+                out_host[b].copy_(dev_out[b], non_blocking=True)
+                ev_down[b].record(s_down)
+        for b in range(NB):
+            ev_down[b].synchronize()
 
-    for i in range(args.warmup):
-        one(i)
+    torch.cuda.synchronize()
+    run(0, max(args.warmup, NB))
+    torch.cuda.synchronize()
     dist.barrier()
     t0 = time.perf_counter()
-    for i in range(args.steps):
-        one(i)
+    run(0, args.steps)
     t = dist.max(time.perf_counter() - t0)
     return {"value": wl.B * dist.world * args.steps / t, "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h}
+            "d2h_bytes_per_step": d2h, "pipelined": "upload of step i+1 and download of step i-1 overlap step i"}
 
 
 # ----------------------------------------------------------------------------- prefill
