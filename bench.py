@@ -167,14 +167,13 @@ def decode_bytes_per_query(wl) -> dict:
     E, k, W, D, H, Hi, Di = wl.E, wl.k, wl.W, wl.D, wl.H, wl.Hi, wl.Di
     keys = E * (Di // 2 + Di // 32)
     qi = Hi * (Di * 4) + Hi * 4           # raw fp32 indexer query + head weights
-    q_fp4 = Hi * (Di // 2 + Di // 32)
     gathered = k * D * 2
     window = W * D * 2
     q_o = 2 * H * D * 2
     idx = k * 4
     score_out = E * 4
     return {"step": keys + qi + gathered + window + q_o + idx,
-            "index_score": keys + q_fp4 + Hi * 4 + score_out,
+            "index_score": keys + Hi * (Di // 2 + Di // 32) + Hi * 4 + score_out,
             "attention": gathered + window + q_o + idx,
             "keys": keys}
 
@@ -196,8 +195,6 @@ def setup_decode(wl, dev, replicas: int):
     torch.cuda.synchronize()
     Bn = wl.B
     ws = {
-        "q_fp4": torch.empty((Bn, wl.Hi, wl.Di // 2), dtype=torch.uint8, device=dev),
-        "q_scale": torch.empty((Bn, wl.Hi, wl.Di // 32), dtype=torch.uint8, device=dev),
         "scores": torch.empty((Bn, wl.E), dtype=torch.float32, device=dev),
         "idx": torch.empty((Bn, wl.k), dtype=torch.int32, device=dev),
         "cnt": torch.empty((Bn,), dtype=torch.int32, device=dev),
@@ -205,12 +202,17 @@ def setup_decode(wl, dev, replicas: int):
         "attn_ws": torch.empty(B.csa_sparse_attn_workspace(Bn, wl.H, wl.D, wl.k, wl.W), dtype=torch.uint8,
                                device=dev),
         "out": torch.empty((Bn, wl.H, wl.D), dtype=torch.bfloat16, device=dev),
+        "q_fp4": torch.empty((Bn, wl.Hi, wl.Di // 2), dtype=torch.uint8, device=dev),
+        "q_scale": torch.empty((Bn, wl.Hi, wl.Di // 32), dtype=torch.uint8, device=dev),
     }
     return caches, steps, ws
 
 
 def decode_step(wl, cache, step, ws, ev=None):
-    """One decode step as four C-ABI calls; `ev` (optional) gets CUDA events between calls."""
+    """One decode step as four C-ABI calls; `ev` (optional) gets CUDA events between calls.
+    (csa_index_score_q would encode the queries inside the indexer instead, but with nine
+    indexer CTAs per query that repeats the encoding nine times; one encoding pass is
+    cheaper here.)"""
     from compressed_sparse_long_02_b200 import binding as B
     if ev is not None:
         ev[0].record()
@@ -305,7 +307,7 @@ def bench_decode(args, dist, peaks):
                           "frac": round(step_gbs / peaks["hbm_gbs"], 4)},
         "per_call_us": {k: round(v * 1e3, 2) for k, v in per.items()},
         "clocks": clk,
-        "gpu_launches": args.steps * 5,  # quantize, index score, top-k, attention, split merge
+        "gpu_launches": args.steps * 4,  # query encoding, indexer, top-k, attention (split merge inside)
         "graph": "one CUDA graph per input replica, replayed back to back",
     }
     res["e2e"] = bench_decode_e2e(args, wl, caches, steps, ws, dist)
@@ -333,10 +335,8 @@ def bench_decode_e2e(args, wl, caches, steps, ws, dist):
     out_host = [torch.empty((wl.B, wl.H, wl.D), dtype=torch.bfloat16).pin_memory() for _ in range(NB)]
     h2d = sum(v.numel() * v.element_size() for v in host[0].values())
     d2h = out_host[0].numel() * out_host[0].element_size()
-    lws = {"q_fp4": ws["q_fp4"], "q_scale": ws["q_scale"], "idx": ws["idx"], "cnt": ws["cnt"], "seq": ws["seq"],
-           "attn_ws": ws["attn_ws"],
-           "index_ws": torch.empty(layer.B.csa_index_topk_workspace(wl.B, wl.E, wl.k), dtype=torch.uint8,
-                                   device=dev)}
+    lws = {"q_fp4": ws["q_fp4"], "q_scale": ws["q_scale"], "scores": ws["scores"], "idx": ws["idx"], "cnt": ws["cnt"],
+           "seq": ws["seq"], "attn_ws": ws["attn_ws"]}
     s_up, s_comp, s_down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev_up = [torch.cuda.Event() for _ in range(NB)]
     ev_comp = [torch.cuda.Event() for _ in range(NB)]

@@ -16,7 +16,7 @@ import threading
 import torch
 
 __all__ = ["CsaError", "lib", "csa_compress", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk",
-           "csa_index_score", "csa_topk_select",
+           "csa_index_score", "csa_index_score_q", "csa_topk_select",
            "csa_index_topk_workspace", "csa_sparse_attn", "csa_sparse_attn_workspace", "hca_attn",
            "hca_attn_workspace", "csa_get_device_error", "LIB_PATH", "DEVERR_NONE", "DEVERR_TIMEOUT",
            "DEVERR_INDEX"]
@@ -54,6 +54,7 @@ def lib() -> ctypes.CDLL:
             L.csa_quantize_mxfp4.argtypes = [P, I, I64, I, P, P, P]
             L.csa_index_topk.argtypes = [I, I, I, I, I, P, P, P, P, P, I, I, P, P, P, P, P, P, P, SZ, P]
             L.csa_index_score.argtypes = [I, I, I, I, P, P, P, P, P, I, I, P, P, P, P, I, P]
+            L.csa_index_score_q.argtypes = [I, I, I, I, P, I, P, P, P, I, I, P, P, P, P, I, P]
             L.csa_topk_select.argtypes = [I, I, I, P, I, P, P, I, I, P, P, P, P]
             L.csa_index_topk_workspace.argtypes = [I, I, I]
             L.csa_index_topk_workspace.restype = SZ
@@ -69,6 +70,7 @@ def lib() -> ctypes.CDLL:
             L.csa_last_cuda_error.argtypes = []
             L.csa_last_cuda_error.restype = ctypes.c_char_p
             for fn in ("csa_compress", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk", "csa_index_score",
+                       "csa_index_score_q",
                        "csa_topk_select", "csa_sparse_attn",
                        "hca_attn", "csa_get_device_error"):
                 getattr(L, fn).restype = I
@@ -212,6 +214,23 @@ def csa_index_score(q_fp4, q_scale, w, q_pos, q_seq, k_fp4, k_scale, n_entries, 
                                E_max, _ptr(k_fp4), _ptr(k_scale), _ptr(n_entries), _ptr(scores), scores.shape[1],
                                _stream(q_fp4))
     _check("csa_index_score", st)
+    return scores
+
+
+def csa_index_score_q(q, w, q_pos, q_seq, k_fp4, k_scale, n_entries, *, m: int,
+                      scores: torch.Tensor | None = None):
+    """csa_index_score with unencoded queries q [Nq, Hi, Di] float32/bf16 (encoded to MXFP4
+    inside the indexer).  Returns scores float32 [Nq, E_stride]."""
+    Nq, Hi, Di = q.shape
+    B, E_max, _ = k_fp4.shape
+    if scores is None:
+        scores = torch.full((Nq, E_max), float("-inf"), dtype=torch.float32, device=q.device)
+    _need(scores, torch.float32, None, "scores")
+    q = q.contiguous()
+    st = lib().csa_index_score_q(Nq, Hi, Di, m, _ptr(q), _dt(q), _ptr(w), _ptr(q_pos), _ptr(q_seq), B, E_max,
+                                 _ptr(k_fp4), _ptr(k_scale), _ptr(n_entries), _ptr(scores), scores.shape[1],
+                                 _stream(q))
+    _check("csa_index_score_q", st)
     return scores
 
 

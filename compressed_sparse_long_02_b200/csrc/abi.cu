@@ -242,6 +242,38 @@ csa_status csa_index_score(int Nq, int Hi, int Di, int m, const uint8_t* q_fp4, 
   return from_cuda(launch_index_score(a, stream));
 }
 
+csa_status csa_index_score_q(int Nq, int Hi, int Di, int m, const void* q, csa_dtype q_dtype, const float* w,
+                             const int32_t* q_pos, const int32_t* q_seq, int B, int E_max, const uint8_t* k_fp4,
+                             const uint8_t* k_scale, const int32_t* n_entries, float* scores, int E_stride,
+                             cudaStream_t stream) {
+  if (Nq < 0 || m < 1 || B < 1 || E_max < 1 || E_stride < E_max) return CSA_ERR_INVALID_ARG;
+  if (q_dtype != CSA_F32 && q_dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
+  if (Hi < 1 || Hi > 64 || (Di != 64 && Di != 128)) return CSA_ERR_UNSUPPORTED;
+  if (E_max % 8 != 0) return CSA_ERR_UNSUPPORTED;
+  if (Nq == 0) return CSA_OK;
+  if (!q || !w || !q_pos || !q_seq || !k_fp4 || !k_scale || !n_entries || !scores) return CSA_ERR_INVALID_ARG;
+  if (!aligned16(k_fp4) || !aligned16(k_scale)) return CSA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(q) & (q_dtype == CSA_F32 ? 7u : 3u)) != 0) return CSA_ERR_ALIGNMENT;
+  IndexArgs a{};
+  a.Nq = Nq;
+  a.Hi = Hi;
+  a.Di = Di;
+  a.m = m;
+  a.B = B;
+  a.E_max = E_max;
+  a.q_raw = q;
+  a.q_raw_bf16 = q_dtype == CSA_BF16 ? 1 : 0;
+  a.w = w;
+  a.q_pos = q_pos;
+  a.q_seq = q_seq;
+  a.k_fp4 = k_fp4;
+  a.k_scale = k_scale;
+  a.n_entries = n_entries;
+  a.scores_ws = scores;
+  a.E_stride = E_stride;
+  return from_cuda(launch_index_score(a, stream));
+}
+
 csa_status csa_topk_select(int Nq, int k, int m, const float* scores, int E_stride, const int32_t* q_pos,
                            const int32_t* q_seq, int B, int E_max, const int32_t* n_entries, int32_t* idx_out,
                            int32_t* cnt_out, cudaStream_t stream) {

@@ -30,6 +30,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "mxfp4.cuh"
 #include "ptx.cuh"
 #include "tmap.h"
 
@@ -56,14 +57,18 @@ struct IndexParams {
   const int32_t* n_entries;
   const uint8_t* q_scale;
   const uint8_t* k_scale;
+  const void* q_raw;  // raw queries [Nq, Hi, Di] (f32 or bf16) when kRawQ: encoded in the kernel
+  int q_raw_bf16;
   float* scores;
   float* score_out;
   int32_t* err;
 };
 
 // kHi: number of indexer heads fixed at compile time (the head chain is straight-line
-// code), or 0 to take it from p.Hi at run time.
-template <int kHi>
+// code), or 0 to take it from p.Hi at run time.  kRawQ: the query arrives unencoded and
+// the epilogue warps encode it to MXFP4 (the same rule as quantize_mxfp4_kernel) into
+// the MMA's B operand and scale factors before the first tile.
+template <int kHi, bool kRawQ>
 __global__ void __launch_bounds__(kIdxThreads, 2)
     index_score_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                        IndexParams p) {
@@ -96,7 +101,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(b_full, 1);
+    mbar_init(b_full, kRawQ ? 8 : 1);
     mbar_init(sf_full, 1);
     mbar_init(sf_ready, 8);
     for (int i = 0; i < kAccBufs; ++i) {
@@ -150,8 +155,10 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
       mbar_arrive_expect_tx(&full[0], a_bytes);
       CSA_T(tslot, 16);
       tma_load_2d(smem_u32(sA), &tm_k, &full[0], 0, row0);
-      mbar_arrive_expect_tx(b_full, b_bytes);
-      tma_load_2d(smem_u32(sB), &tm_q, b_full, 0, q * Hi);
+      if (!kRawQ) {
+        mbar_arrive_expect_tx(b_full, b_bytes);
+        tma_load_2d(smem_u32(sB), &tm_q, b_full, 0, q * Hi);
+      }
       // entries with a scale byte in the cache: E_max and tile starts are multiples of 8,
       // so the byte count is a multiple of 16
       const int sf_entries = min(n_tiles * kTileE, p.E_max - t_begin * kTileE);
@@ -172,7 +179,12 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
     // ------------------------------------------------------------ MMA issuer
     // scale factors of B (the query's heads) into the tcgen05 scale-factor layout:
     // row r -> byte (r % 32) * 16 + (r / 32) * 4 + block; rows >= Hi are zero (2^-127)
-    {
+    if (kRawQ) {
+      // the epilogue warps encoded the query into sB and sSFB
+      const bool got = warp_wait(b_full, 0, p.err, abort_flag);
+      if (got && lane == 0) tc_cp_32x128b_warpx4(tmem + kColSFB, smem_desc(smem_u32(sSFB), 0, 128, kSwizzleNone));
+      __syncwarp();
+    } else {
       uint32_t words[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -227,6 +239,49 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
     if (ew * 32 + lane < 64) {
       const int h = ew * 32 + lane;
       sW[h] = h < Hi ? __ldg(p.w + static_cast<size_t>(q) * Hi + h) : 0.f;
+    }
+    if (kRawQ) {
+      // Encode the query (Hi rows x Di) into the B operand: K-major, the 16-byte chunk c of
+      // row h at h * row_bytes + ((c ^ swizzle(h)) << 4) (SWIZZLE_64B: (h >> 1) & 3 for
+      // 64-byte rows; SWIZZLE_32B: (h >> 2) & 1 for 32-byte rows), and its scale bytes
+      // into the scale-factor layout.  Rows past Hi (N is a multiple of 16) stay zero.
+      const int te = threadIdx.x - 64;  // 0..255
+      for (int i = te; i < 128; i += 256) reinterpret_cast<uint32_t*>(sSFB)[i] = 0u;
+      for (int i = Hi * row_bytes / 4 + te; i < p.N * row_bytes / 4; i += 256) reinterpret_cast<uint32_t*>(sB)[i] = 0u;
+      named_bar_sync(1, 256);
+      const int pairs = Hi * row_bytes;  // element pairs = FP4 bytes; a multiple of 16, <= 4096
+      const size_t qbase = static_cast<size_t>(q) * Hi * p.Di;
+      constexpr int kPer = 64 * 64 / 256;  // pairs per thread at most
+      float2 xv[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {  // every load in flight before any encoding
+        const int g = te + 256 * i;
+        xv[i] = make_float2(0.f, 0.f);
+        if (g < pairs) {
+          if (p.q_raw_bf16) {
+            const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.q_raw) + qbase) + g);
+            xv[i] = make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+          } else {
+            xv[i] = __ldg(reinterpret_cast<const float2*>(static_cast<const float*>(p.q_raw) + qbase) + g);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int g = te + 256 * i;
+        if (g - lane >= pairs) break;  // warp-uniform: whole warps past the end
+        uint8_t byte, sbyte;
+        mxfp4_encode_pair(xv[i].x, xv[i].y, byte, sbyte);
+        if (g < pairs) {
+          const int h = g / row_bytes, b = g % row_bytes;
+          const int sw = row_bytes == 64 ? (h >> 1) & 3 : (h >> 2) & 1;
+          sB[h * row_bytes + (((b >> 4) ^ sw) << 4) + (b & 15)] = byte;
+          if ((b & 15) == 0) sSFB[(h % 32) * 16 + (h / 32) * 4 + (b >> 4)] = sbyte;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_full);
     }
     // key scales: entry-major bytes -> scale-factor layout, warp ew takes tiles ew, ew + 8, ...
     // (word (r % 32) * 4 + r / 32 of a 512-byte slot holds the scale bytes of entry r)
@@ -297,7 +352,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
   }
 }
 
-int g_index_smem[2][64];
+int g_index_smem[4][64];
 
 }  // namespace
 
@@ -313,7 +368,10 @@ cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s) {
   const CUtensorMapSwizzle swz = row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   if (!encode_2d_u8(&tm_k, a.k_fp4, row_bytes, static_cast<uint64_t>(a.B) * a.E_max, row_bytes, kTileE, swz))
     return cudaErrorInvalidValue;
-  if (!encode_2d_u8(&tm_q, a.q_fp4, row_bytes, static_cast<uint64_t>(a.Nq) * a.Hi, row_bytes, N, swz))
+  // raw queries are encoded in the kernel: the query map is then unused (any valid map)
+  if (!(a.q_raw != nullptr
+            ? encode_2d_u8(&tm_q, a.k_fp4, row_bytes, static_cast<uint64_t>(a.B) * a.E_max, row_bytes, N, swz)
+            : encode_2d_u8(&tm_q, a.q_fp4, row_bytes, static_cast<uint64_t>(a.Nq) * a.Hi, row_bytes, N, swz)))
     return cudaErrorInvalidValue;
 
   IndexParams p{};
@@ -341,14 +399,16 @@ cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s) {
   p.err = device_error_word();
 
   const size_t smem = 1024 + kStages * 8192 + 4096 + kMaxTilesPerCta * (512 + 256) + 512 + 256 + 512;
-  if (a.Hi == 64) {
-    cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(index_score_kernel<64>), smem, g_index_smem[0]);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(index_score_kernel<64>, dim3(a.Nq * p.splits), dim3(kIdxThreads), smem, s, tm_k, tm_q, p);
-  }
-  cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(index_score_kernel<0>), smem, g_index_smem[1]);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(index_score_kernel<0>, dim3(a.Nq * p.splits), dim3(kIdxThreads), smem, s, tm_k, tm_q, p);
+  p.q_raw = a.q_raw;
+  p.q_raw_bf16 = a.q_raw_bf16;
+  const dim3 grid(a.Nq * p.splits), block(kIdxThreads);
+  auto go = [&](auto kern, int slot) -> cudaError_t {
+    const cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(kern), smem, g_index_smem[slot]);
+    return e != cudaSuccess ? e : launch_pdl(kern, grid, block, smem, s, tm_k, tm_q, p);
+  };
+  if (a.q_raw != nullptr)
+    return a.Hi == 64 ? go(index_score_kernel<64, true>, 2) : go(index_score_kernel<0, true>, 3);
+  return a.Hi == 64 ? go(index_score_kernel<64, false>, 0) : go(index_score_kernel<0, false>, 1);
 }
 
 }  // namespace csa

@@ -86,6 +86,8 @@ struct IndexArgs {
   int Nq, Hi, Di, k, m, B, E_max;
   const uint8_t* q_fp4;
   const uint8_t* q_scale;
+  const void* q_raw;  // non-null: unencoded queries [Nq, Hi, Di], encoded to MXFP4 in the indexer
+  int q_raw_bf16;
   const float* w;
   const int32_t* q_pos;
   const int32_t* q_seq;

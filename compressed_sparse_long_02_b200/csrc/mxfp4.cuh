@@ -23,16 +23,21 @@ __device__ __forceinline__ int mx_block_exponent(float amax) {
   return E < -127 ? -127 : (E > 127 ? 127 : E);
 }
 
-__device__ __forceinline__ uint32_t e2m1_code(float x, int E) {
-  const float a = fabsf(ldexpf(x, -E));
-  const uint32_t c = a <= 0.25f   ? 0u
-                     : a < 0.75f  ? 1u
-                     : a <= 1.25f ? 2u
-                     : a < 1.75f  ? 3u
-                     : a <= 2.5f  ? 4u
-                     : a < 3.5f   ? 5u
-                     : a <= 5.0f  ? 6u
-                                  : 7u;
+// 2^E as a float, E in [-127, 127] (2^-127 is the subnormal 0x00400000)
+__device__ __forceinline__ float mx_pow2(int E) {
+  return E >= -126 ? __uint_as_float(static_cast<uint32_t>(E + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// E2M1 code of x / 2^E, taken as comparisons of |x| against the rounding boundaries
+// scaled by T = 2^E (products by powers of two, all representable): the same decision
+// as rounding |x| / 2^E half-to-even onto {0, .5, 1, 1.5, 2, 3, 4, 6}, without forming
+// the quotient.  Bit 3 is the sign of x.
+__device__ __forceinline__ uint32_t e2m1_code(float x, float T) {
+  const float a = fabsf(x);
+  uint32_t c = (a > 0.25f * T ? 1u : 0u) + (a >= 0.75f * T ? 1u : 0u) + (a > 1.25f * T ? 1u : 0u) +
+               (a >= 1.75f * T ? 1u : 0u) + (a > 2.5f * T ? 1u : 0u) + (a >= 3.5f * T ? 1u : 0u) +
+               (a > 5.0f * T ? 1u : 0u);
+  if (a == INFINITY) c = 7u;  // the scaled boundaries overflow only when T = 2^127
   return c | (signbit(x) ? 8u : 0u);
 }
 
@@ -43,7 +48,8 @@ __device__ __forceinline__ void mxfp4_encode_pair(float x0, float x1, uint8_t& b
 #pragma unroll
   for (int o = 1; o < 16; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
   const int E = mx_block_exponent(am);
-  byte = static_cast<uint8_t>(e2m1_code(x0, E) | (e2m1_code(x1, E) << 4));
+  const float T = mx_pow2(E);
+  byte = static_cast<uint8_t>(e2m1_code(x0, T) | (e2m1_code(x1, T) << 4));
   scale_byte = static_cast<uint8_t>(E + 127);
 }
 

@@ -204,6 +204,17 @@ CSA_API csa_status csa_index_score(int Nq, int Hi, int Di, int m, const uint8_t*
                                    const float* w, const int32_t* q_pos, const int32_t* q_seq, int B, int E_max,
                                    const uint8_t* k_fp4, const uint8_t* k_scale, const int32_t* n_entries,
                                    float* scores, int E_stride, cudaStream_t stream);
+/*
+ * csa_index_score_q -- csa_index_score taking the indexer queries unencoded:
+ * q [Nq, Hi, Di] in q_dtype (CSA_F32 or CSA_BF16), row-major, 8-byte aligned (f32) or
+ * 4-byte aligned (bf16).  Each query is encoded to MXFP4 inside the indexer by the rule
+ * of csa_quantize_mxfp4 (same bytes), so the scores equal csa_quantize_mxfp4 followed by
+ * csa_index_score; the encoded query is not written out.  Same support limits.
+ */
+CSA_API csa_status csa_index_score_q(int Nq, int Hi, int Di, int m, const void* q, csa_dtype q_dtype, const float* w,
+                                     const int32_t* q_pos, const int32_t* q_seq, int B, int E_max,
+                                     const uint8_t* k_fp4, const uint8_t* k_scale, const int32_t* n_entries,
+                                     float* scores, int E_stride, cudaStream_t stream);
 CSA_API csa_status csa_topk_select(int Nq, int k, int m, const float* scores, int E_stride, const int32_t* q_pos,
                                    const int32_t* q_seq, int B, int E_max, const int32_t* n_entries,
                                    int32_t* idx_out, int32_t* cnt_out, cudaStream_t stream);

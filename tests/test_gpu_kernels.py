@@ -175,6 +175,35 @@ def test_index_topk_decode_multi_sequence(B, cuda):
     _err_clear(B)
 
 
+@pytest.mark.parametrize("Hi,Di,dtype", [(64, 128, "f32"), (64, 128, "bf16"), (4, 64, "f32"), (20, 128, "bf16")])
+def test_index_score_q_encodes_inside(B, cuda, Hi, Di, dtype):
+    """Unencoded queries: the indexer's own MXFP4 encoding gives the oracle's scores bit for bit."""
+    rng = np.random.default_rng(31 + Hi + Di)
+    Bq, E = 3, 2048
+    ki = rng.standard_normal((Bq, E, Di)).astype(np.float32)
+    kp, ks = oracle.mxfp4_quantize(ki)
+    qi = (rng.standard_normal((Bq, Hi, Di)) * rng.choice([1e-3, 1.0, 40.0], (Bq, Hi, 1))).astype(np.float32)
+    if dtype == "bf16":
+        bits = synth.to_dtype_np(qi, "bf16")
+        q_dev = to_dev_bf16(bits, cuda)
+        qi = bf16_bits_to_f64(bits).astype(np.float32)
+    else:
+        q_dev = to_dev(qi, cuda)
+    qp, qs = oracle.mxfp4_quantize(qi)
+    w = rng.uniform(0, 1, (Bq, Hi)).astype(np.float32)
+    n_ent = np.array([E, 1500, 777], np.int32)
+    pos = (n_ent.astype(np.int64) * 4 - 1).astype(np.int32)
+    seqs = np.arange(Bq, dtype=np.int32)
+    n_vis = np.array([oracle.n_visible(pos[b], 4, n_ent[b]) for b in range(Bq)], np.int32)
+    s32, _, bad = oracle.index_scores(qp, qs, w, seqs, n_vis, kp, ks)
+    assert bad == 0
+    sc = t2np(B.csa_index_score_q(q_dev, to_dev(w, cuda), to_dev(pos, cuda), to_dev(seqs, cuda), to_dev(kp, cuda),
+                                  to_dev(ks, cuda), to_dev(n_ent, cuda), m=4))
+    for b in range(Bq):
+        np.testing.assert_array_equal(sc[b, :n_vis[b]], s32[b, :n_vis[b]])
+    _err_clear(B)
+
+
 def test_topk_ties_lowest_index(B, cuda):
     """All keys identical: every score ties, the k lowest indices must win."""
     Hi, Di, E, k = 8, 128, 1024, 100
