@@ -26,8 +26,9 @@
 // thread and are reduced once at the end.
 //
 // Roles (416 threads): warps 0-7 softmax + epilogue, warps 8-11 gather producers
-// (cp.async, 16-byte chunks; Q arrives by TMA), warp 12 TMEM owner and MMA issuer.  When a query's keys are split over several CTAs
-// (few queries), the splits of a query form a thread-block cluster: each CTA writes an
+// (cp.async, 16-byte chunks; Q arrives by TMA), warp 12 TMEM owner and MMA issuer.
+// When a query's keys are split over several CTAs (few queries), the splits of a
+// query form a thread-block cluster: each CTA writes an
 // unnormalised fp32 partial and its (max, sum) to the workspace, the cluster
 // synchronises, and CTA r combines heads [r H/S, (r+1) H/S) of the query.
 #include <cuda_bf16.h>
@@ -272,6 +273,11 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     const int ptid = threadIdx.x - 256;
     const int r0 = kRowsPerProd * pw;
     const int nrows = min(kRowsPerProd, kBN - r0);
+    if (ptid == 0) {
+      // query: 64 head rows x 1 KB as 8 boxes of 64 rows x 128 B (one per 64-dim atom)
+      mbar_arrive_expect_tx(q_full, kH * kD * 2);
+      for (int a = 0; a < 8; ++a) tma_load_2d(smem_u32(sQ + a * 8192), &tm_q, q_full, 128 * a, n * kH);
+    }
     // this CTA's slice of the index list, staged once per warp (no dependent global load
     // per row); each warp copies the part its own lanes will read
     const int sel_here = max(0, min(row_end, kl.n_sel) - row_begin);
@@ -281,12 +287,6 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
         if ((i % kBN) >= r0 && (i % kBN) < r0 + nrows)
           sidx[i] = p.idx[static_cast<size_t>(n) * p.k + row_begin + i];
     __syncwarp();
-    if (ptid == 0) {
-      prefetch_tmap(&tm_q);
-      // query: 64 head rows x 1 KB as 8 boxes of 64 rows x 128 B (one per 64-dim atom)
-      mbar_arrive_expect_tx(q_full, kH * kD * 2);
-      for (int a = 0; a < 8; ++a) tma_load_2d(smem_u32(sQ + a * 8192), &tm_q, q_full, 128 * a, n * kH);
-    }
     // source row of this lane in a tile (nullptr: no row; invalid indices are flagged once)
     auto row_src = [&](int tile, bool flag) -> const uint16_t* {
       const int g = row_begin + tile * kBN + r0 + lane;
@@ -543,8 +543,10 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
       if (t == 0 && hh == 0 && it < 8) CSA_T(tslot, 48 + it);
     }
     // ------------------------------------------------------------ epilogue
+    CSA_TB(6);
     const bool fin_ok = !named_bar_or(1, 256, !mbar_wait(fin, 0, p.err, abort_flag));  // all 256 take part
     ok = ok && fin_ok;
+    CSA_TB(7);
     if (t == 0 && hh == 0) CSA_T(tslot, 2);
     tc_fence_after();
     xreduce32<false>(lacc);  // lane holds head h0+lane summed over this warp's 32 keys
@@ -691,6 +693,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
   // memory before the reads below.
   __threadfence();
   cluster_sync_all();
+  CSA_TB(4);
   const int S = p.splits;
   const int hp = kH / S;            // heads this CTA combines
   const int hb = split * hp;
@@ -714,24 +717,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     if (p.lse) p.lse[n * kH + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
   }
   __syncthreads();
-  // hp heads x 512 dims, 4 dims per item
+  // hp heads x 512 dims, 4 dims per item; every partial an item needs is loaded before
+  // any is used (the loads come from L2 and would otherwise run one after another)
   for (int it = threadIdx.x; it < hp * (kD / 4); it += blockDim.x) {
     const int hl = it / (kD / 4), d4 = it % (kD / 4);
     const int h = hb + hl;
+    float4 v[kMaxSplits];
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s)
+      v[s] = s < S ? __ldcg(reinterpret_cast<const float4*>(
+                                p.part_o + ((static_cast<size_t>(n) * S + s) * kH + h) * kD) + d4)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < S; ++s) {
-      const float w = wsm[hl * S + s];
-      if (w == 0.f) continue;
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(
-                                  p.part_o + ((static_cast<size_t>(n) * S + s) * kH + h) * kD) + d4);
-      acc.x = fmaf(v.x, w, acc.x);
-      acc.y = fmaf(v.y, w, acc.y);
-      acc.z = fmaf(v.z, w, acc.z);
-      acc.w = fmaf(v.w, w, acc.w);
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {
+      const float w = s < S ? wsm[hl * S + s] : 0.f;
+      if (w == 0.f) continue;  // an empty split's partial is never read as a number
+      acc.x = fmaf(v[s].x, w, acc.x);
+      acc.y = fmaf(v[s].y, w, acc.y);
+      acc.z = fmaf(v[s].z, w, acc.z);
+      acc.w = fmaf(v[s].w, w, acc.w);
     }
     uint2 o2 = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
     *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(n) * kH + h) * kD + 4 * d4) = o2;
   }
+  CSA_TB(5);
 }
 
 int g_attn_smem[64];

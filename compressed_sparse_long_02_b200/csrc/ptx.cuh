@@ -22,7 +22,7 @@
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                       \
     if ((slot) >= 0 && (slot) < 64 && (ev) >= 0 && (ev) < 64) g_csa_timing[slot][ev] = t_; \
   } while (0)
-// CSA_TB(ev): per-CTA stamp into g_csa_cta[1024][4] (first 1024 CTAs), same builds only
+// CSA_TB(ev): per-CTA stamp into g_csa_cta[1024][8] (first 1024 CTAs), same builds only
 #define CSA_TB(ev)                                                               \
   do {                                                                           \
     unsigned long long t_;                                                       \
@@ -68,6 +68,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test: has the phase of `bar` with parity `parity` completed?
+__device__ __forceinline__ bool mbar_test(const uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
