@@ -170,15 +170,6 @@ __device__ __forceinline__ void stage_of(int st, int n_tiles, int& tile, bool& i
   }
 }
 
-// every thread of every CTA in the cluster; release / acquire order global memory too
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
 
 // Shared-memory layout of a CTA (one definition for the set-up and the pipeline).
 struct AttnSmem {
@@ -805,21 +796,8 @@ cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s) {
   }
   cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(attn_kernel), kAttnSmem, g_attn_smem);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.Nq * splits);
-  cfg.blockDim = dim3(kAttnThreads);
-  cfg.dynamicSmemBytes = kAttnSmem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = static_cast<unsigned>(splits);
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, attn_kernel, tm_q, p);
+  return launch_pdl_cluster(attn_kernel, dim3(a.Nq * splits), dim3(kAttnThreads), kAttnSmem,
+                            static_cast<unsigned>(splits), s, tm_q, p);
 }
 
 }  // namespace csa

@@ -295,6 +295,42 @@ __device__ __forceinline__ void griddep_enter() {
   griddep_trigger();
 }
 
+// ------------------------------------------------------------------ thread-block clusters
+// Every thread of every CTA in the cluster takes part; the release / acquire pair orders
+// shared and global memory writes before the barrier with reads after it, cluster-wide.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_sync_all() {
+  cluster_arrive();
+  cluster_wait();
+}
+// address in the shared::cluster window of the object at `p` (this CTA's shared memory)
+// in the shared memory of cluster CTA `rank`
+__device__ __forceinline__ uint32_t dsmem_map(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// Loads from another CTA's shared memory take several hundred cycles; callers issue all
+// of them before using any (the asm is ordered after earlier barriers by `volatile`, but
+// carries no memory clobber, so independent loads stay in flight together).
+__device__ __forceinline__ uint32_t dsmem_ld(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint2 dsmem_ld2(uint32_t addr) {  // 8-byte aligned
+  uint2 v;
+  asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint4 dsmem_ld4(uint32_t addr) {  // 16-byte aligned
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
 // ------------------------------------------------------------------ misc
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 

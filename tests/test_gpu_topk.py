@@ -2,11 +2,13 @@
 
 The same float32 score rows go to both sides, so index sets must be identical (no tie
 exemption: ties resolve to the lowest index on both sides).  Cases span every kernel
-variant -- rows held in registers (16 / 32 entries per thread, rows up to 2048, 8192
-and 32768 entries) and rows staged in shared memory (longer rows, read from global
-memory beyond its capacity) -- with ragged visible counts, rows at or below k, exact
-ties across warp boundaries, -0/+0, negative scores, an outlier that crowds the
-threshold bin (the digit-pass path), and a score stride wider than E_max.
+variant -- rows held in the registers of a thread-block cluster of 2, 4 or 8 CTAs (few
+rows: 8, 16 or 32 entries per thread), of one CTA (many rows: 16 / 32 entries per
+thread, rows up to 2048, 8192 and 32768 entries), and rows staged in shared memory
+(longer rows, read from global memory beyond its capacity) -- with ragged visible
+counts, rows at or below k, exact ties across warp and CTA boundaries, -0/+0, negative
+scores, an outlier that crowds the threshold bin (the digit-pass path), and a score
+stride wider than E_max.
 """
 import numpy as np
 import pytest
@@ -65,6 +67,30 @@ def test_topk_row_lengths(B, cuda, E, k, kind):
     s = _rows(kind, Nq, E, rng)
     n_vis = rng.integers(0, E + 1, Nq).astype(np.int32)
     n_vis[:6] = [E, k, k + 1, 0, 1, E - 1]
+    _run(B, cuda, s, n_vis, k, E)
+
+
+@pytest.mark.parametrize("E,k", [(2000, 256), (8000, 1024), (30000, 1024)])
+@pytest.mark.parametrize("kind", ["normal", "levels", "outlier"])
+def test_topk_many_rows(B, cuda, E, k, kind):
+    """160 rows: more rows than a wave of clusters, so one CTA per row holds it."""
+    rng = np.random.default_rng(300 + E)
+    Nq = 160
+    s = _rows(kind, Nq, E, rng)
+    n_vis = rng.integers(0, E + 1, Nq).astype(np.int32)
+    n_vis[:5] = [E, k, k + 1, 0, E - 1]
+    _run(B, cuda, s, n_vis, k, E)
+
+
+@pytest.mark.parametrize("Nq,E", [(4, 262144), (8, 100000), (16, 65536)])
+def test_topk_cluster_of_eight(B, cuda, Nq, E):
+    """Few long rows: eight CTAs per row, up to 32 entries per thread (the 1M-token decode shape)."""
+    rng = np.random.default_rng(400 + Nq)
+    k = 1024
+    s = _rows("normal", Nq, E, rng)
+    s[0, E // 8 - 700:E // 8 + 700] = 6.5     # a tie group across the first CTA boundary
+    n_vis = np.full(Nq, E, np.int32)
+    n_vis[-1] = E - 12345
     _run(B, cuda, s, n_vis, k, E)
 
 
