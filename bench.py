@@ -435,9 +435,37 @@ def bench_prefill(name, steps, warmup, dist, peaks):
                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                         "frac": round(tf / peaks["bf16_tflops_sustained"], 4), "attention_ms": round(attn_ms, 4),
                         "algorithmic_flops": flops}}
+    if wl.kind == "csa_prefill":
+        # the indexer's scoring alone: MXFP4 contraction of every visible (query, entry) pair
+        scores = torch.empty((wl.T, r["k_fp4"].shape[1]), dtype=torch.float32, device=dev)
+        for _ in range(2):
+            B.csa_index_score(r["q_fp4"], r["q_scale"], r["w"], pos, seq, r["k_fp4"], r["k_scale"], r["n_ent"], m=wl.m,
+                              scores=scores)
+        i0, i1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        i0.record()
+        for _ in range(reps):
+            B.csa_index_score(r["q_fp4"], r["q_scale"], r["w"], pos, seq, r["k_fp4"], r["k_scale"], r["n_ent"], m=wl.m,
+                              scores=scores)
+        i1.record()
+        torch.cuda.synchronize()
+        idx_ms = i0.elapsed_time(i1) / reps
+        iflops = indexer_flops(wl)
+        itf = iflops / (idx_ms / 1e3) / 1e12
+        fp4_peak = peaks["bf16_tflops"] * 4.0  # nominal dense fp4 / bf16 ratio (9 / 2.25) on the measured burst
+        out["indexer"] = {"bound": "tensor", "kernel": "index_score", "achieved": round(itf, 1),
+                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(itf / fp4_peak, 4),
+                          "index_ms": round(idx_ms, 4), "algorithmic_flops": iflops,
+                          "peak_source": "measured bf16 burst x 4 (nominal MXFP4 / bf16 ratio)"}
+        del scores
     del t, r
     torch.cuda.empty_cache()
     return out
+
+
+def indexer_flops(wl) -> float:
+    """2 x Hi x Di over every visible (query, entry) pair the indexer scores."""
+    tot = sum(min((t + 1) // wl.m, wl.E) for t in range(wl.T))
+    return 2.0 * wl.Hi * wl.Di * tot
 
 
 def attention_flops(wl) -> float:

@@ -22,6 +22,10 @@
 //               taking alternate tiles: one thread per entry (TMEM lane), ReLU,
 //               head-weighted fp32 chain, store of the score
 // Barrier set-up and the TMEM allocation run before the wait on the previous grid.
+//
+// index_score_persistent_kernel (below) serves many queries of the common shape
+// (Hi = 64, Di = 128): persistent CTAs take blocks of eight queries and load each key
+// tile once per block.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -352,7 +356,373 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
   }
 }
 
-int g_index_smem[4][64];
+// ---------------------------------------------------------------------- many queries
+// index_score_persistent_kernel -- Hi = 64, Di = 128, many queries (prefill).  Queries are
+// taken in blocks of eight consecutive ones.  One persistent CTA per SM deals itself
+// blocks heaviest first in a zigzag over the grid (causal rows grow with position), and
+// loads every key tile a block needs once for all of its queries: each tile feeds four
+// N = 128 MMAs, one per pair of queries (an N = 128 block-scaled MMA costs what an N = 64
+// one does), so the key stream is an eighth of one pass per query.
+//   warp 0       producer: per block the eight queries' FP4 rows (TMA), scale bytes and
+//                head weights (bulk copies) into one of two block buffers; per tile 128
+//                FP4 key rows (TMA, SWIZZLE_64B) and their scale bytes (bulk copy)
+//   warp 1       MMA: per block the pairs' scale bytes into the tcgen05 scale-factor
+//                layout and TMEM; per tile the keys' (a 32 x 4 word transpose in place),
+//                then per pair two kind::mxf4.block_scale MMAs (M = 128 entries, N = 128 =
+//                two queries' heads, K = 64 each) into one of three accumulators
+//   warps 2..25  epilogue: group g of eight warps drains accumulator g, two warps per TMEM
+//                lane quarter (one per query of the pair); one thread per entry: ReLU,
+//                head-weighted fp32 chain, store
+// A block whose queries span several sequences runs as segments, one per sequence run,
+// each with its own key tiles; the pairs a segment touches compute both halves and keep
+// the segment's queries.  Every role derives the same (segment, tile, pair) order.
+constexpr int kPStages = 10;
+constexpr int kBlkQ = 8;               // queries per block
+constexpr int kPairs = kBlkQ / 2;      // N = 128 MMAs per key tile
+constexpr int kPAcc = 3;               // accumulators of 128 columns
+constexpr int kPGroups = kPAcc;        // epilogue group g drains accumulator g
+constexpr int kPEpiWarps = 8;          // per group: 4 lane quarters x 2 queries
+constexpr int kPThreads = 32 * (2 + kPEpiWarps * kPGroups);
+constexpr uint32_t kPTmemCols = 512;
+constexpr uint32_t kPColSFA = 128 * kPAcc;              // ring of kSfRing x 4 columns
+constexpr uint32_t kPColSFB = kPColSFA + 4 * kSfRing;   // 2 blocks x kPairs x 4 columns
+static_assert(kPColSFB + 2 * kPairs * 4 <= kPTmemCols, "TMEM budget (one CTA per SM)");
+
+// The eight queries of block b: validity, sequence, visible entries, and the segments
+// (maximal runs of valid queries sharing a sequence, in query order).
+struct BlockInfo {
+  int nseg;
+  int seq[kBlkQ], nvis[kBlkQ];
+  uint32_t valid;            // bit g: query 8b + g exists and has a sequence in range
+  int seg_seq[kBlkQ], seg_lo[kBlkQ], seg_hi[kBlkQ], seg_nt[kBlkQ];
+};
+
+__device__ __forceinline__ void block_info(const IndexParams& p, int b, BlockInfo& bi) {
+  bi.valid = 0;
+  bi.nseg = 0;
+#pragma unroll
+  for (int g = 0; g < kBlkQ; ++g) {
+    const int q = b * kBlkQ + g;
+    bi.seq[g] = -1;
+    bi.nvis[g] = 0;
+    if (q < p.Nq) {
+      const int s = p.q_seq[q];
+      if (s >= 0 && s < p.B) {
+        bi.seq[g] = s;
+        bi.nvis[g] = min(visible_entries(p.q_pos[q], p.m, p.n_entries[s]), p.E_max);
+        bi.valid |= 1u << g;
+      }
+    }
+  }
+  for (int g = 0; g < kBlkQ; ++g) {
+    if (!(bi.valid >> g & 1u)) continue;
+    const int nt = (bi.nvis[g] + kTileE - 1) / kTileE;
+    if (bi.nseg > 0 && bi.seg_seq[bi.nseg - 1] == bi.seq[g]) {
+      bi.seg_hi[bi.nseg - 1] = g;
+      bi.seg_nt[bi.nseg - 1] = max(bi.seg_nt[bi.nseg - 1], nt);
+    } else {
+      bi.seg_seq[bi.nseg] = bi.seq[g];
+      bi.seg_lo[bi.nseg] = g;
+      bi.seg_hi[bi.nseg] = g;
+      bi.seg_nt[bi.nseg] = nt;
+      ++bi.nseg;
+    }
+  }
+}
+
+struct PersistSmem {
+  uint8_t* sA;     // kPStages x 8 KB key tiles (1024-aligned)
+  uint8_t* sSFA;   // kPStages x 512: a tile's scale bytes (raw, then scale-factor layout)
+  uint8_t* sB;     // 2 x kBlkQ x 4 KB query rows (1024-aligned); pair p = 8 KB at 8 KB p
+  uint8_t* sSFB;   // 2 x kBlkQ x 256 raw scale bytes; pair p's 512 B become its layout
+  float* sW;       // 2 x kBlkQ x 64 head weights
+  BlockInfo* info; // 2: the block in each buffer, written by the producer
+  uint64_t* full;       // [kPStages]
+  uint64_t* empty;      // [kPStages]
+  uint64_t* blk_full;   // [2]
+  uint64_t* blk_empty;  // [2]
+  uint64_t* acc_full;   // [kPAcc]
+  uint64_t* acc_empty;  // [kPAcc]
+  uint64_t* fin;
+  uint32_t* tmem_slot;
+  volatile int* abort_flag;
+  __device__ explicit PersistSmem(uint8_t* s) {
+    sA = s;
+    sSFA = sA + kPStages * 8192;
+    sB = sSFA + kPStages * 512;
+    sSFB = sB + 2 * kBlkQ * 4096;
+    sW = reinterpret_cast<float*>(sSFB + 2 * kBlkQ * 256);
+    info = reinterpret_cast<BlockInfo*>(sW + 2 * kBlkQ * 64);
+    full = reinterpret_cast<uint64_t*>(info + 2);
+    empty = full + kPStages;
+    blk_full = empty + kPStages;
+    blk_empty = blk_full + 2;
+    acc_full = blk_empty + 2;
+    acc_empty = acc_full + kPAcc;
+    fin = acc_empty + kPAcc;
+    tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+    abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  }
+};
+constexpr size_t kPersistSmem = 1024 + kPStages * (8192 + 512) + 2 * kBlkQ * (4096 + 256 + 256) +
+                                2 * sizeof(BlockInfo) + 8 * (2 * kPStages + 4 + 2 * kPAcc + 1) + 16;
+static_assert(sizeof(BlockInfo) % 8 == 0, "barriers after the block infos stay 8-byte aligned");
+static_assert(kPersistSmem <= 227 * 1024, "shared memory budget");
+
+// block dealt to this CTA in round r (zigzag over the grid, heaviest blocks first), or -1
+__device__ __forceinline__ int dealt_block(int r, int nblk) {
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const int k = r * G + ((r & 1) ? (G - 1 - c) : c);
+  return k < nblk ? nblk - 1 - k : -1;
+}
+
+// In place: 128 words of row-major scale bytes (word r = the 4 scale bytes of row r) ->
+// the scale-factor layout of a 32x128b copy (word 4 (r % 32) + r / 32).  Rows at or past
+// `rows` are zero.  All 32 lanes of the warp call it.
+__device__ __forceinline__ void sf_transpose(uint8_t* buf, int rows, int lane) {
+  uint32_t* w = reinterpret_cast<uint32_t*>(buf);
+  uint32_t v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = lane + 32 * i < rows ? w[lane + 32 * i] : 0u;
+  __syncwarp();
+  reinterpret_cast<uint4*>(buf)[lane] = make_uint4(v[0], v[1], v[2], v[3]);
+}
+
+__global__ void __launch_bounds__(kPThreads, 1)
+    index_score_persistent_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                                  IndexParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const PersistSmem L(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kHiP = 64;
+  constexpr uint32_t kSbo = 8 * 64;  // 8-row SWIZZLE_64B atom of 64-byte rows
+  const int nblk = (p.Nq + kBlkQ - 1) / kBlkQ;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(&L.full[s], 1);
+      mbar_init(&L.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&L.blk_full[b], 1);
+      mbar_init(&L.blk_empty[b], 1 + kPEpiWarps * kPGroups);  // the MMA thread's commit, then each epilogue warp
+    }
+    for (int i = 0; i < kPAcc; ++i) {
+      mbar_init(&L.acc_full[i], 1);
+      mbar_init(&L.acc_empty[i], kPEpiWarps);
+    }
+    mbar_init(L.fin, 1);
+    *L.abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_q);
+  }
+  if (warp == 1) {
+    tmem_alloc(L.tmem_slot, kPTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *L.tmem_slot;
+  griddep_enter();
+  volatile int* abort_flag = L.abort_flag;
+  const bool stamp = blockIdx.x == 0;  // development timing builds: CTA 0's pipeline events
+  if (stamp && threadIdx.x == 0) CSA_T(9, 0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      int T = 0;
+      BlockInfo bi;
+      for (int r = 0; ok; ++r) {  // blocks alternate between the two buffers, empty ones too
+        const int b = dealt_block(r, nblk);
+        if (b < 0) break;
+        block_info(p, b, bi);
+        for (int g = 0; g < kBlkQ; ++g)  // sequence ids out of range produce nothing
+          if (b * kBlkQ + g < p.Nq && !(bi.valid >> g & 1u)) atomicExch(p.err, CSA_DEVERR_INDEX);
+        const int bb = r & 1;
+        if (!mbar_wait(&L.blk_empty[bb], ((r >> 1) & 1) ^ 1, p.err, abort_flag)) break;
+        if (stamp && r < 64) CSA_T(15, r);
+        L.info[bb] = bi;  // published by the arrival below
+        mbar_arrive_expect_tx(&L.blk_full[bb], __popc(bi.valid) * (4096 + 256 + 256));
+        for (int g = 0; g < kBlkQ; ++g) {
+          if (!(bi.valid >> g & 1u)) continue;
+          const int q = b * kBlkQ + g;
+          const int slot = bb * kBlkQ + g;
+          tma_load_2d(smem_u32(L.sB + slot * 4096), &tm_q, &L.blk_full[bb], 0, q * kHiP);
+          bulk_load(smem_u32(L.sSFB + slot * 256), p.q_scale + static_cast<size_t>(q) * kHiP * 4, 256, &L.blk_full[bb]);
+          bulk_load(smem_u32(L.sW + slot * 64), p.w + static_cast<size_t>(q) * kHiP, 256, &L.blk_full[bb]);
+        }
+        for (int sg = 0; ok && sg < bi.nseg; ++sg) {
+          for (int j = 0; j < bi.seg_nt[sg]; ++j, ++T) {
+            const int st = T % kPStages;
+            if (!mbar_wait(&L.empty[st], ((T / kPStages) & 1) ^ 1, p.err, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const int e0 = j * kTileE;
+            const int row0 = bi.seg_seq[sg] * p.E_max + e0;
+            // scale bytes of the entries the cache holds (E_max and e0 are multiples of 8)
+            const uint32_t sf_bytes = static_cast<uint32_t>(min(kTileE, p.E_max - e0) * 4);
+            if (stamp && T < 64) CSA_T(10, T);
+            mbar_arrive_expect_tx(&L.full[st], 8192 + sf_bytes);
+            tma_load_2d(smem_u32(L.sA + st * 8192), &tm_k, &L.full[st], 0, row0);
+            bulk_load(smem_u32(L.sSFA + st * 512), p.k_scale + static_cast<size_t>(row0) * 4, sf_bytes, &L.full[st]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA
+    bool ok = true;
+    int T = 0, U = 0;
+    for (int r = 0; ok; ++r) {
+      if (dealt_block(r, nblk) < 0) break;
+      const int bb = r & 1;
+      ok = warp_wait_sleep(&L.blk_full[bb], (r >> 1) & 1, p.err, abort_flag);
+      if (!ok) break;
+      const BlockInfo& bi = L.info[bb];
+      if (bi.nseg == 0) {
+        if (lane == 0) mbar_arrive(&L.blk_empty[bb]);
+        __syncwarp();
+        continue;
+      }
+      if (stamp && lane == 0 && r < 64) CSA_T(16, r);
+#pragma unroll 1
+      for (int pr = 0; pr < kPairs; ++pr) sf_transpose(L.sSFB + (bb * kBlkQ + 2 * pr) * 256, 128, lane);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tc_fence_after();
+        for (int pr = 0; pr < kPairs; ++pr)
+          tc_cp_32x128b_warpx4(tmem + kPColSFB + 4 * (bb * kPairs + pr),
+                               smem_desc(smem_u32(L.sSFB + (bb * kBlkQ + 2 * pr) * 256), 0, 128, kSwizzleNone));
+      }
+      __syncwarp();
+      for (int sg = 0; ok && sg < bi.nseg; ++sg) {
+        const int p_lo = bi.seg_lo[sg] >> 1, p_hi = bi.seg_hi[sg] >> 1;
+        for (int j = 0; ok && j < bi.seg_nt[sg]; ++j, ++T) {
+          const int st = T % kPStages;
+          ok = warp_wait_sleep(&L.full[st], (T / kPStages) & 1, p.err, abort_flag);
+          if (!ok) break;
+          if (stamp && lane == 0 && T < 64) CSA_T(11, T);
+          sf_transpose(L.sSFA + st * 512, min(kTileE, p.E_max - j * kTileE), lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tc_fence_after();
+            const uint32_t sfa = tmem + kPColSFA + 4 * (T % kSfRing);
+            tc_cp_32x128b_warpx4(sfa, smem_desc(smem_u32(L.sSFA + st * 512), 0, 128, kSwizzleNone));
+            const uint32_t a0 = smem_u32(L.sA + st * 8192);
+            for (int pr = p_lo; ok && pr <= p_hi; ++pr, ++U) {
+              const int buf = U % kPAcc;
+              ok = mbar_wait_sleep(&L.acc_empty[buf], ((U / kPAcc) & 1) ^ 1, p.err, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+              const uint32_t b0 = smem_u32(L.sB + (bb * kBlkQ + 2 * pr) * 4096);
+              const uint32_t sfb = tmem + kPColSFB + 4 * (bb * kPairs + pr);
+#pragma unroll
+              for (int kh = 0; kh < 2; ++kh) {
+                const uint32_t sf_id = 2 * kh;  // byte of the scale column holding blocks 2kh, 2kh+1
+                mma_mxf4(tmem + 128 * buf, smem_desc(a0 + 32 * kh, 0, kSbo, kSwizzle64B),
+                         smem_desc(b0 + 32 * kh, 0, kSbo, kSwizzle64B), idesc_mxf4(kTileE, 2 * kHiP, sf_id, sf_id),
+                         kh > 0 ? 1u : 0u, sfa | (sf_id << 30), sfb | (sf_id << 30));
+              }
+              tc_commit(&L.acc_full[buf]);
+            }
+            tc_commit(&L.empty[st]);  // the key tile's last MMA has read it
+            if (stamp && T < 64) CSA_T(12, T);
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          U = __shfl_sync(0xffffffffu, U, 0);
+        }
+      }
+      if (lane == 0 && ok) tc_commit(&L.blk_empty[bb]);  // the block's MMAs no longer read its buffer
+      __syncwarp();
+    }
+    if (lane == 0) {  // every tcgen05 operation of this thread (and its commits) has completed
+      tc_commit(L.fin);
+      volatile int never = 0;
+      mbar_wait(L.fin, 0, p.err, &never);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..25)
+    const int grp = (warp - 2) / kPEpiWarps;  // accumulator this group drains
+    const int half = ((warp - 2) % kPEpiWarps) >> 2;  // query of the pair: 2 pr + half
+    const int sub = warp & 3;                 // TMEM lane quarter this warp may access
+    const uint32_t lane_base = static_cast<uint32_t>(32 * sub) << 16;
+    bool ok = true;
+    int U = 0;
+    for (int r = 0; ok; ++r) {
+      const int b = dealt_block(r, nblk);
+      if (b < 0) break;
+      const int bb = r & 1;
+      ok = warp_wait_sleep(&L.blk_full[bb], (r >> 1) & 1, p.err, abort_flag);  // the block and its head weights
+      const BlockInfo& bi = L.info[bb];
+      for (int sg = 0; ok && sg < bi.nseg; ++sg) {
+        const int p_lo = bi.seg_lo[sg] >> 1, p_hi = bi.seg_hi[sg] >> 1;
+        const int s_seq = bi.seg_seq[sg];
+        for (int j = 0; ok && j < bi.seg_nt[sg]; ++j) {
+          for (int pr = p_lo; ok && pr <= p_hi; ++pr, ++U) {
+            if (U % kPAcc != grp) continue;
+            ok = warp_wait_sleep(&L.acc_full[grp], (U / kPAcc) & 1, p.err, abort_flag);
+            if (!ok) break;
+            if (stamp && sub == 0 && half == 0 && lane == 0 && U < 64) CSA_T(13, U);
+            tc_fence_after();
+            const int g = 2 * pr + half;
+            const bool keep = (bi.valid >> g & 1u) && bi.seq[g] == s_seq && g >= bi.seg_lo[sg] && g <= bi.seg_hi[sg];
+            const float* w = L.sW + (bb * kBlkQ + g) * 64;
+            const uint32_t taddr = tmem + lane_base + 128 * grp + 64 * half;
+            float s = 0.f;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {  // 32 heads per TMEM read
+              uint32_t x[32];
+              tmem_ld16(taddr + 32 * c, x);
+              tmem_ld16(taddr + 32 * c + 16, x + 16);
+              tmem_wait_ld();
+              if (c == 1) {  // the accumulator is read: the next MMA may overwrite it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&L.acc_empty[grp]);
+              }
+#pragma unroll
+              for (int hh = 0; hh < 32; hh += 4) {
+                const float4 w4 = *reinterpret_cast<const float4*>(w + 32 * c + hh);
+                s = fmaf(w4.x, fmaxf(__uint_as_float(x[hh]), 0.f), s);
+                s = fmaf(w4.y, fmaxf(__uint_as_float(x[hh + 1]), 0.f), s);
+                s = fmaf(w4.z, fmaxf(__uint_as_float(x[hh + 2]), 0.f), s);
+                s = fmaf(w4.w, fmaxf(__uint_as_float(x[hh + 3]), 0.f), s);
+              }
+            }
+            const int e = j * kTileE + 32 * sub + lane;
+            if (keep && e < bi.nvis[g]) {
+              const int q = b * kBlkQ + g;
+              p.scores[static_cast<size_t>(q) * p.E_stride + e] = s;
+              if (p.score_out) p.score_out[static_cast<size_t>(q) * p.E_max + e] = s;
+            }
+            if (stamp && sub == 0 && half == 0 && lane == 0 && U < 64) CSA_T(14, U);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&L.blk_empty[bb]);  // done with the block's weights
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kPTmemCols);
+  }
+}
+
+int g_index_smem[5][64];
 
 }  // namespace
 
@@ -397,6 +767,18 @@ cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s) {
   p.scores = a.scores_ws;
   p.score_out = a.score_out;
   p.err = device_error_word();
+
+  // many pre-encoded queries of the common shape: persistent CTAs, several queries each
+  if (a.q_raw == nullptr && a.Hi == 64 && a.Di == 128 && a.Nq >= 2 * num_sms() &&
+      (reinterpret_cast<uintptr_t>(a.w) & 15u) == 0 && (reinterpret_cast<uintptr_t>(a.q_scale) & 15u) == 0 &&
+      (reinterpret_cast<uintptr_t>(a.k_scale) & 15u) == 0) {
+    const cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(index_score_persistent_kernel), kPersistSmem,
+                                       g_index_smem[4]);
+    if (e != cudaSuccess) return e;
+    const int nblk = (a.Nq + kBlkQ - 1) / kBlkQ;
+    return launch_pdl(index_score_persistent_kernel, dim3(std::min(nblk, num_sms())), dim3(kPThreads), kPersistSmem,
+                      s, tm_k, tm_q, p);
+  }
 
   const size_t smem = 1024 + kStages * 8192 + 4096 + kMaxTilesPerCta * (512 + 256) + 512 + 256 + 512;
   p.q_raw = a.q_raw;

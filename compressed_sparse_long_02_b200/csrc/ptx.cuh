@@ -103,6 +103,42 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
   }
 }
 
+// The same wait for roles with many waiting warps: try_wait carries a suspend-time hint,
+// so a waiting thread sleeps until the phase completes (or 1 ms passes) instead of
+// polling the barrier and the abort flag, which would take shared-memory bandwidth from
+// the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(1000000u)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, int32_t* err,
+                                                volatile int* abort_flag) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait_sleep(a, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait_sleep(a, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicExch(err, CSA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool warp_wait_sleep(uint64_t* bar, uint32_t parity, int32_t* err,
+                                                volatile int* abort_flag) {
+  const bool ok = mbar_wait_sleep(bar, parity, err, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // All 32 lanes wait; every lane gets the same answer (false if any lane gave up), so
 // the warp stays converged for the collectives that follow.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int32_t* err, volatile int* abort_flag) {

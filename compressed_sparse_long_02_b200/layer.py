@@ -48,7 +48,7 @@ def csa_prefill(wl, t: dict, rows: torch.Tensor | None = None) -> dict:
     out, lse = B.csa_sparse_attn(q, pos, seq, pool["entries"], idx, cnt, pool["window"], _i32([0], dev), W=wl.W,
                                  want_lse=True)
     return dict(out=out, lse=lse, idx=idx, cnt=cnt, entries=pool["entries"], window=pool["window"],
-                k_fp4=keys["fp4"], k_scale=keys["fp4_scale"], q=q, q_fp4=q_fp4, q_scale=q_sc)
+                k_fp4=keys["fp4"], k_scale=keys["fp4_scale"], q=q, q_fp4=q_fp4, q_scale=q_sc, w=w, n_ent=n_ent)
 
 
 def csa_decode(wl, cache: dict, step: dict, ws: dict | None = None, out: torch.Tensor | None = None) -> dict:

@@ -136,8 +136,11 @@ def _index_case(wl, T, rows, dev, B):
                 n_vis=n_vis, E=E)
 
 
-@pytest.mark.parametrize("name,T,nrows", [("tiny", 512, None), ("csa_prefill_8k", 2048, 160)])
+@pytest.mark.parametrize("name,T,nrows", [("tiny", 512, None), ("csa_prefill_8k", 2048, 160),
+                                         ("csa_prefill_8k", 2048, None), ("csa_prefill_8k", 8192, 400)])
 def test_index_topk_exact(B, cuda, name, T, nrows):
+    """Scores bit-exact and index sets exact; 2048 and ~400 rows reach the persistent
+    many-query indexer (at least two queries per SM), 160 rows the per-query one."""
     wl = synth.WORKLOADS[name]
     rng = np.random.default_rng(9)
     if nrows is None:
@@ -173,6 +176,38 @@ def test_index_topk_decode_multi_sequence(B, cuda):
         np.testing.assert_array_equal(sc[b, :n_vis[b]], s32[b, :n_vis[b]])
     check_topk(t2np(idx), t2np(cnt), idx_r, cnt_r, kth, s32, n_vis, wl.k)
     _err_clear(B)
+
+
+def test_index_score_many_queries_multi_sequence(B, cuda):
+    """400 queries over 3 sequences with ragged entry counts (the persistent indexer): scores
+    bit-exact on every visible entry, the rest of each row untouched; rows whose sequence id
+    is out of range are left alone and flag CSA_DEVERR_INDEX."""
+    rng = np.random.default_rng(77)
+    Bs, E_max, Hi, Di, m = 3, 1024, 64, 128, 4
+    n_ent = np.array([1024, 777, 1000], np.int32)
+    kp, ks = oracle.mxfp4_quantize(rng.standard_normal((Bs, E_max, Di)).astype(np.float32))
+    Nq = 400
+    seq = rng.integers(0, Bs, Nq).astype(np.int32)
+    seq[[5, 200, 399]] = [-1, 3, -1]
+    pos = (rng.integers(0, 4 * E_max + 40, Nq)).astype(np.int32)
+    pos[:4] = [0, 3, 4 * 777 - 1, 4 * 1024 + 39]
+    qp, qs = oracle.mxfp4_quantize(rng.standard_normal((Nq, Hi, Di)).astype(np.float32))
+    w = rng.random((Nq, Hi)).astype(np.float32)
+    ok = (seq >= 0) & (seq < Bs)
+    n_vis = np.array([oracle.n_visible(int(pos[i]), m, int(n_ent[seq[i]])) if ok[i] else 0 for i in range(Nq)],
+                     np.int32)
+    s32, _, bad = oracle.index_scores(qp[ok], qs[ok], w[ok], seq[ok], n_vis[ok], kp, ks)
+    assert bad == 0
+    sentinel = np.float32(-7.25)
+    scores = to_dev(np.full((Nq, E_max + 4), sentinel, np.float32), cuda)
+    B.csa_index_score(to_dev(qp, cuda), to_dev(qs, cuda), to_dev(w, cuda), to_dev(pos, cuda), to_dev(seq, cuda),
+                      to_dev(kp, cuda), to_dev(ks, cuda), to_dev(n_ent, cuda), m=m, scores=scores)
+    sc = t2np(scores)
+    ref = np.full_like(sc, sentinel)
+    vis = np.arange(E_max)[None, :] < n_vis[ok][:, None]
+    ref[np.where(ok)[0], :E_max] = np.where(vis, s32, sentinel)
+    np.testing.assert_array_equal(sc, ref)
+    assert B.csa_get_device_error() == B.DEVERR_INDEX  # read and cleared
 
 
 @pytest.mark.parametrize("Hi,Di,dtype", [(64, 128, "f32"), (64, 128, "bf16"), (4, 64, "f32"), (20, 128, "bf16")])
