@@ -53,12 +53,12 @@ def load_peaks() -> dict:
 # decode step (profiles/*_decode_128k.md), keyed by the sha1 of the kernel's source file
 # at capture time: a kernel changed since its capture reports traffic null.
 NCU_TRAFFIC = {
-    "attention": {"bytes": 40267520 + 761600, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
-                  "sha1": "67a07667369369326db30edc16e072746dca66f2"},
-    "index_score": {"bytes": 71479808 + 1585408, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
-                    "sha1": "0d868836e8e3b78c9d584e62b4bc2ac54fe9f374"},
-    "topk_select": {"bytes": 4260352, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",
-                    "sha1": "ef5746a9441cc408c3142e9e9c2489cef61a1b1e"},
+    "attention": {"bytes": 40078592 + 838912, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
+                  "sha1": "d04f12d89dfa6efd041251fb20408de5cf6134a9"},
+    "index_score": {"bytes": 71479552 + 1724928, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
+                    "sha1": "92645beee700a6035b78e2d12283f92df90069dd"},
+    "topk_select": {"bytes": 4252672, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",
+                    "sha1": "58b7e4b5c9975a744f5b58160cfdafb4cf85ff3c"},
 }
 
 
