@@ -551,24 +551,30 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     named_bar_sync(1, 256);
     if (ok) {
 #pragma unroll 1
-      for (int dc = 0; dc < 4; ++dc) {
-        uint32_t o[32];
-        const uint32_t ta = tmem + lane_base + kColO + 64 * dc + h0;
-        tmem_ld16(ta, o);
-        tmem_ld16(ta + 16, o + 16);
+      for (int dp = 0; dp < 4; dp += 2) {  // two 128-dim chunks per TMEM round trip
+        uint32_t o[2][32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t ta = tmem + lane_base + kColO + 64 * (dp + c) + h0;
+          tmem_ld16(ta, o[c]);
+          tmem_ld16(ta + 16, o[c] + 16);
+        }
         tmem_wait_ld();
-        const int d = dc * 128 + t;
-        if (p.splits == 1) {
-          uint16_t* ob = p.out + (static_cast<size_t>(n) * kH + h0) * kD + d;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const __nv_bfloat16 bv = __float2bfloat16_rn(__uint_as_float(o[i]) * inv_l[h0 + i]);
-            ob[i * kD] = *reinterpret_cast<const uint16_t*>(&bv);
+        for (int c = 0; c < 2; ++c) {
+          const int d = (dp + c) * 128 + t;
+          if (p.splits == 1) {
+            uint16_t* ob = p.out + (static_cast<size_t>(n) * kH + h0) * kD + d;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const __nv_bfloat16 bv = __float2bfloat16_rn(__uint_as_float(o[c][i]) * inv_l[h0 + i]);
+              ob[i * kD] = *reinterpret_cast<const uint16_t*>(&bv);
+            }
+          } else {
+            float* pbo = p.part_o + ((static_cast<size_t>(n) * p.splits + split) * kH + h0) * kD + d;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pbo[i * kD] = __uint_as_float(o[c][i]);
           }
-        } else {
-          float* pbo = p.part_o + ((static_cast<size_t>(n) * p.splits + split) * kH + h0) * kD + d;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) pbo[i * kD] = __uint_as_float(o[i]);
         }
       }
       if (threadIdx.x < kH) {
@@ -635,6 +641,46 @@ __device__ __forceinline__ uint32_t attn_setup(uint8_t* smem) {
   __syncthreads();
   tc_fence_after();
   return *tmem_slot;
+}
+
+// The combine step of a query split S ways: heads [hb, hb + 64 / S) x 512 dims, 4 dims
+// per item, weights wsm[hl * S + s] (zero for a split that contributes nothing).  A
+// thread's items are it = threadIdx.x + j blockDim.x; every partial of every item of the
+// thread is loaded before any is used (about 20 loads from L2 in flight per thread
+// instead of one round trip per item).
+template <int S>
+__device__ __forceinline__ void merge_partials(const AttnParams& p, int n, int hb, const float* wsm) {
+  constexpr int kItems = kH / S * (kD / 4);
+  constexpr int kPer = (kItems + kAttnThreads - 1) / kAttnThreads;  // items per thread at most
+  float4 v[kPer][S];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int it = static_cast<int>(threadIdx.x) + j * kAttnThreads;
+    const int hl = it / (kD / 4), d4 = it % (kD / 4);
+#pragma unroll
+    for (int s = 0; s < S; ++s)
+      v[j][s] = it < kItems ? __ldcg(reinterpret_cast<const float4*>(
+                                  p.part_o + ((static_cast<size_t>(n) * S + s) * kH + hb + hl) * kD) + d4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int it = static_cast<int>(threadIdx.x) + j * kAttnThreads;
+    if (it >= kItems) break;
+    const int hl = it / (kD / 4), d4 = it % (kD / 4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      const float w = wsm[hl * S + s];
+      if (w == 0.f) continue;  // an empty split's partial is never read as a number
+      acc.x = fmaf(v[j][s].x, w, acc.x);
+      acc.y = fmaf(v[j][s].y, w, acc.y);
+      acc.z = fmaf(v[j][s].z, w, acc.z);
+      acc.w = fmaf(v[j][s].w, w, acc.w);
+    }
+    const uint2 o2 = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+    *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(n) * kH + hb + hl) * kD + 4 * d4) = o2;
+  }
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_constant__ CUtensorMap tm_q, AttnParams p) {
@@ -708,29 +754,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     if (p.lse) p.lse[n * kH + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
   }
   __syncthreads();
-  // hp heads x 512 dims, 4 dims per item; every partial an item needs is loaded before
-  // any is used (the loads come from L2 and would otherwise run one after another)
-  for (int it = threadIdx.x; it < hp * (kD / 4); it += blockDim.x) {
-    const int hl = it / (kD / 4), d4 = it % (kD / 4);
-    const int h = hb + hl;
-    float4 v[kMaxSplits];
-#pragma unroll
-    for (int s = 0; s < kMaxSplits; ++s)
-      v[s] = s < S ? __ldcg(reinterpret_cast<const float4*>(
-                                p.part_o + ((static_cast<size_t>(n) * S + s) * kH + h) * kD) + d4)
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int s = 0; s < kMaxSplits; ++s) {
-      const float w = s < S ? wsm[hl * S + s] : 0.f;
-      if (w == 0.f) continue;  // an empty split's partial is never read as a number
-      acc.x = fmaf(v[s].x, w, acc.x);
-      acc.y = fmaf(v[s].y, w, acc.y);
-      acc.z = fmaf(v[s].z, w, acc.z);
-      acc.w = fmaf(v[s].w, w, acc.w);
-    }
-    uint2 o2 = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-    *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(n) * kH + h) * kD + 4 * d4) = o2;
+  if (S == 2) {
+    merge_partials<2>(p, n, hb, wsm);
+  } else if (S == 4) {
+    merge_partials<4>(p, n, hb, wsm);
+  } else {
+    merge_partials<kMaxSplits>(p, n, hb, wsm);
   }
   CSA_TB(5);
 }
