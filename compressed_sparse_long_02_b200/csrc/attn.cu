@@ -644,12 +644,12 @@ __device__ __forceinline__ uint32_t attn_setup(uint8_t* smem) {
 }
 
 // The combine step of a query split S ways: heads [hb, hb + 64 / S) x 512 dims, 4 dims
-// per item, weights wsm[hl * S + s] (zero for a split that contributes nothing).  A
-// thread's items are it = threadIdx.x + j blockDim.x; every partial of every item of the
-// thread is loaded before any is used (about 20 loads from L2 in flight per thread
-// instead of one round trip per item).
+// per item.  A thread's items are it = threadIdx.x + j blockDim.x; every partial of every
+// item of the thread is loaded before any is used (about 20 loads from L2 in flight per
+// thread instead of one round trip per item), and the per-head weights (shared memory
+// wsm[hl * S + s], zero for a split that contributes nothing) are formed meanwhile.
 template <int S>
-__device__ __forceinline__ void merge_partials(const AttnParams& p, int n, int hb, const float* wsm) {
+__device__ __forceinline__ void merge_partials(const AttnParams& p, int n, int hb, float* wsm) {
   constexpr int kItems = kH / S * (kD / 4);
   constexpr int kPer = (kItems + kAttnThreads - 1) / kAttnThreads;  // items per thread at most
   float4 v[kPer][S];
@@ -663,6 +663,30 @@ __device__ __forceinline__ void merge_partials(const AttnParams& p, int n, int h
                                   p.part_o + ((static_cast<size_t>(n) * S + s) * kH + hb + hl) * kD) + d4)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  // while those are in flight: per head, each split's (max, sum) in one round trip, the
+  // weights 2^(m_s - M) / L with L = sum_s l_s 2^(m_s - M), and the log-sum-exp
+  if (static_cast<int>(threadIdx.x) < kH / S) {
+    const int h = hb + static_cast<int>(threadIdx.x);
+    float2 ml[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) ml[s] = __ldcg(&p.part_ml[(static_cast<size_t>(n) * S + s) * kH + h]);
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < S; ++s)
+      if (ml[s].y > 0.f) M = fmaxf(M, ml[s].x);
+    float w[S];
+    float L = 0.f;
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      w[s] = ml[s].y > 0.f ? exp2f(ml[s].x - M) : 0.f;
+      L = fmaf(ml[s].y, w[s], L);
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int s = 0; s < S; ++s) wsm[threadIdx.x * S + s] = w[s] * inv;
+    if (p.lse) p.lse[n * kH + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+  }
+  __syncthreads();
 #pragma unroll
   for (int j = 0; j < kPer; ++j) {
     const int it = static_cast<int>(threadIdx.x) + j * kAttnThreads;
@@ -734,26 +758,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
   const int S = p.splits;
   const int hp = kH / S;            // heads this CTA combines
   const int hb = split * hp;
-  float* wsm = reinterpret_cast<float*>(smem);  // [hp][S] weights / L, then [hp] lse
-  if (static_cast<int>(threadIdx.x) < hp) {
-    const int h = hb + threadIdx.x;
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) {
-      const float2 ml = p.part_ml[(static_cast<size_t>(n) * S + s) * kH + h];
-      if (ml.y > 0.f) M = fmaxf(M, ml.x);
-    }
-    float L = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float2 ml = p.part_ml[(static_cast<size_t>(n) * S + s) * kH + h];
-      const float w = ml.y > 0.f ? exp2f(ml.x - M) : 0.f;
-      wsm[threadIdx.x * S + s] = w;
-      L = fmaf(ml.y, w, L);
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    for (int s = 0; s < S; ++s) wsm[threadIdx.x * S + s] *= inv;
-    if (p.lse) p.lse[n * kH + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
-  }
-  __syncthreads();
+  float* wsm = reinterpret_cast<float*>(smem);  // [hp][S] weights / L
   if (S == 2) {
     merge_partials<2>(p, n, hb, wsm);
   } else if (S == 4) {
