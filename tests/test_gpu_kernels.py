@@ -179,9 +179,10 @@ def test_index_topk_decode_multi_sequence(B, cuda):
 
 
 def test_index_score_many_queries_multi_sequence(B, cuda):
-    """400 queries over 3 sequences with ragged entry counts (the persistent indexer): scores
-    bit-exact on every visible entry, the rest of each row untouched; rows whose sequence id
-    is out of range are left alone and flag CSA_DEVERR_INDEX."""
+    """400 queries over 3 sequences with ragged entry counts (the persistent indexer, whose
+    blocks of eight queries then span several sequences): scores bit-exact on every visible
+    entry, the rest of each row untouched; rows whose sequence id is out of range, one
+    whole block of them included, are left alone and flag CSA_DEVERR_INDEX."""
     rng = np.random.default_rng(77)
     Bs, E_max, Hi, Di, m = 3, 1024, 64, 128, 4
     n_ent = np.array([1024, 777, 1000], np.int32)
@@ -189,6 +190,7 @@ def test_index_score_many_queries_multi_sequence(B, cuda):
     Nq = 400
     seq = rng.integers(0, Bs, Nq).astype(np.int32)
     seq[[5, 200, 399]] = [-1, 3, -1]
+    seq[16:24] = -1                              # a whole block of eight queries without a sequence
     pos = (rng.integers(0, 4 * E_max + 40, Nq)).astype(np.int32)
     pos[:4] = [0, 3, 4 * 777 - 1, 4 * 1024 + 39]
     qp, qs = oracle.mxfp4_quantize(rng.standard_normal((Nq, Hi, Di)).astype(np.float32))
