@@ -15,7 +15,7 @@ import threading
 
 import torch
 
-__all__ = ["CsaError", "lib", "csa_compress", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk",
+__all__ = ["CsaError", "lib", "csa_compress", "csa_compress_step", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk",
            "csa_index_score", "csa_index_score_q", "csa_topk_select",
            "csa_index_topk_workspace", "csa_sparse_attn", "csa_sparse_attn_workspace", "hca_attn",
            "hca_attn_workspace", "csa_get_device_error", "LIB_PATH", "DEVERR_NONE", "DEVERR_TIMEOUT",
@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
             L = ctypes.CDLL(LIB_PATH)
             P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
             L.csa_compress.argtypes = [ctypes.POINTER(_PoolCfg), I, I, P, P, P, P, I, P, P, P, P]
+            L.csa_compress_step.argtypes = [ctypes.POINTER(_PoolCfg), I, P, P, P, P, P, I, P, P, P]
             L.csa_norm_rope.argtypes = [P, I, I64, I, I, P, I64, I, F, I, F, P, P]
             L.csa_quantize_mxfp4.argtypes = [P, I, I64, I, P, P, P]
             L.csa_index_topk.argtypes = [I, I, I, I, I, P, P, P, P, P, I, I, P, P, P, P, P, P, P, SZ, P]
@@ -69,7 +70,7 @@ def lib() -> ctypes.CDLL:
             L.csa_status_string.restype = ctypes.c_char_p
             L.csa_last_cuda_error.argtypes = []
             L.csa_last_cuda_error.restype = ctypes.c_char_p
-            for fn in ("csa_compress", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk", "csa_index_score",
+            for fn in ("csa_compress", "csa_compress_step", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk", "csa_index_score",
                        "csa_index_score_q",
                        "csa_topk_select", "csa_sparse_attn",
                        "hca_attn", "csa_get_device_error"):
@@ -141,6 +142,26 @@ def csa_compress(kv: torch.Tensor, logits: torch.Tensor, slot_bias: torch.Tensor
                             _ptr(out["window"]), _stream(kv))
     _check("csa_compress", st)
     return out
+
+
+def csa_compress_step(kv: torch.Tensor, logits: torch.Tensor, slot_bias: torch.Tensor, pos: torch.Tensor, *, m: int,
+                      overlap: bool, norm: bool, eps: float = 1e-6, rope_dims: int = 0, theta: float = 10000.0,
+                      entries: torch.Tensor | None = None, fp4: torch.Tensor | None = None,
+                      fp4_scale: torch.Tensor | None = None):
+    """Decode-time compressor: kv/logits [B, (1+overlap)*m, C] hold each sequence's last raw
+    tokens (row s = token pos - S + 1 + s); writes the entry that token pos completes into
+    entries [B, E_max, C] (bf16) and / or fp4 [B, E_max, C/2] + fp4_scale [B, E_max, C/32]."""
+    B, S, C = kv.shape
+    assert S == (2 if overlap else 1) * m, "kv must hold the last (1 + overlap) * m tokens"
+    _need(slot_bias, torch.float32, (S, C), "slot_bias")
+    _need(pos, torch.int32, (B,), "pos")
+    ref = entries if entries is not None else fp4
+    assert ref is not None, "nothing to write"
+    E_max = ref.shape[1]
+    cfg = _PoolCfg(m, int(bool(overlap)), C, int(bool(norm)), eps, rope_dims, theta, _dt(kv))
+    st = lib().csa_compress_step(ctypes.byref(cfg), B, _ptr(pos), _ptr(kv.contiguous()), _ptr(logits.contiguous()),
+                                 _ptr(slot_bias), _ptr(entries), E_max, _ptr(fp4), _ptr(fp4_scale), _stream(kv))
+    _check("csa_compress_step", st)
 
 
 def csa_norm_rope(x: torch.Tensor, pos: torch.Tensor | None, *, norm: bool, eps: float = 1e-6, rope_dims: int = 0,

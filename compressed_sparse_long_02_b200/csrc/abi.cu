@@ -134,6 +134,45 @@ csa_status csa_compress(const csa_pool_cfg* cfg, int B, int T, const void* kv, c
   return from_cuda(launch_norm_rope(w, stream));
 }
 
+csa_status csa_compress_step(const csa_pool_cfg* cfg, int B, const int32_t* pos, const void* kv, const void* logits,
+                             const float* slot_bias, void* entries, int E_max, uint8_t* fp4_out, uint8_t* fp4_scale,
+                             cudaStream_t stream) {
+  if (cfg == nullptr || B < 0 || cfg->m < 1 || cfg->m > 128 || (cfg->overlap != 0 && cfg->overlap != 1))
+    return CSA_ERR_INVALID_ARG;
+  if (cfg->rope_dims < 0 || (cfg->rope_dims & 1) || cfg->rope_dims > cfg->C) return CSA_ERR_INVALID_ARG;
+  if (cfg->in_dtype != CSA_F32 && cfg->in_dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
+  if (!pow2_channels(cfg->C)) return CSA_ERR_UNSUPPORTED;
+  if ((fp4_out == nullptr) != (fp4_scale == nullptr)) return CSA_ERR_INVALID_ARG;
+  if (B == 0) return CSA_OK;
+  if (pos == nullptr || kv == nullptr || logits == nullptr || slot_bias == nullptr || E_max < 1)
+    return CSA_ERR_INVALID_ARG;
+  if (!aligned16(kv) || !aligned16(logits) || !aligned16(slot_bias) || !aligned16(entries) || !aligned16(fp4_out) ||
+      !aligned16(fp4_scale))
+    return CSA_ERR_ALIGNMENT;
+  PoolArgs a{};
+  a.kv = kv;
+  a.logits = logits;
+  a.in_bf16 = cfg->in_dtype == CSA_BF16;
+  a.bias = slot_bias;
+  a.B = B;
+  a.T = 0;
+  a.C = cfg->C;
+  a.m = cfg->m;
+  a.overlap = cfg->overlap;
+  a.norm = cfg->norm;
+  a.eps = cfg->eps;
+  a.rope_dims = cfg->rope_dims;
+  a.theta = cfg->rope_theta;
+  a.entries = static_cast<uint16_t*>(entries);
+  a.E_max = E_max;
+  a.fp4 = fp4_out;
+  a.fp4_scale = fp4_scale;
+  a.pos = pos;
+  a.err = device_error_word();
+  if (a.err == nullptr) return CSA_ERR_CUDA;
+  return from_cuda(launch_pool(a, stream));
+}
+
 csa_status csa_norm_rope(const void* x, csa_dtype dtype, int64_t rows, int heads, int C, const int32_t* pos,
                          int64_t pos_mod, int norm, float eps, int rope_dims, float rope_theta, void* out,
                          cudaStream_t stream) {

@@ -64,22 +64,36 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return t;
 }
 
-// one CTA = `epc` consecutive entries of one sequence; thread = channel pair
+// one CTA = `epc` consecutive entries of one sequence; thread = channel pair.  In
+// streaming mode (a.pos set) a CTA serves one sequence and writes at most the one entry
+// its newest token completes, from the sequence's last S raw rows.
 template <bool kBf16>
 __global__ void pool_kernel(PoolArgs a, int epc) {
   griddep_enter();
   __shared__ float red[32];
   const int b = blockIdx.y;
-  const int E = a.T / a.m;
   const int C = a.C;
   const int c0 = 2 * threadIdx.x;
   const int S = a.overlap ? 2 * a.m : a.m;
+  const bool stream = a.pos != nullptr;
+  int E = a.T / a.m, j_stream = 0, tok_ring = 0;
+  if (stream) {  // uniform over the CTA
+    const int pos = a.pos[b];
+    if (pos < 0 || (pos + 1) % a.m != 0) return;  // no group completes at this token
+    j_stream = (pos + 1) / a.m - 1;
+    if (j_stream >= a.E_max) {
+      if (threadIdx.x == 0) atomicExch(a.err, CSA_DEVERR_INDEX);
+      return;
+    }
+    tok_ring = pos - S + 1;  // token of ring row 0
+    E = j_stream + 1;
+  }
   const int rope_base = C - a.rope_dims;
   const bool rot = a.rope_dims > 0 && c0 >= rope_base;
   const double inv_freq = rot ? pow(static_cast<double>(a.theta), -2.0 * ((c0 - rope_base) / 2) / a.rope_dims) : 0.0;
 
   for (int jj = 0; jj < epc; ++jj) {
-    const int j = blockIdx.x * epc + jj;
+    const int j = stream ? j_stream : blockIdx.x * epc + jj;
     if (j >= E) break;  // uniform over the CTA
     const int first = a.overlap ? a.m * (j - 1) : a.m * j;
     float mx0 = -INFINITY, mx1 = -INFINITY, den0 = 0.f, den1 = 0.f, num0 = 0.f, num1 = 0.f;
@@ -87,7 +101,8 @@ __global__ void pool_kernel(PoolArgs a, int epc) {
     for (int s = 0; s < S; ++s) {
       const int tok = first + s;
       if (tok < 0) continue;  // previous group of entry 0 does not exist: excluded
-      const size_t off = (static_cast<size_t>(b) * a.T + tok) * C + c0;
+      const size_t row = stream ? static_cast<size_t>(b) * S + (tok - tok_ring) : static_cast<size_t>(b) * a.T + tok;
+      const size_t off = row * C + c0;
       const float2 x = load_pair<kBf16>(a.kv, off);
       const float2 z = load_pair<kBf16>(a.logits, off);
       const float2 bs = __ldg(reinterpret_cast<const float2*>(a.bias + static_cast<size_t>(s) * C + c0));
@@ -138,6 +153,7 @@ __global__ void pool_kernel(PoolArgs a, int epc) {
       }
       reinterpret_cast<uint32_t*>(a.entries)[eoff / 2] = pack_bf16x2(e0, e1);
     }
+    if (stream) break;
   }
 }
 
@@ -216,8 +232,14 @@ cudaError_t launch_norm_rope(const NormRopeArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s) {
+  if (a.entries == nullptr && a.fp4 == nullptr) return cudaSuccess;
+  if (a.pos != nullptr) {  // streaming: one CTA per sequence
+    const dim3 grid(1, a.B), block(a.C / 2);
+    return a.in_bf16 ? launch_pdl(pool_kernel<true>, grid, block, 0, s, a, 1)
+                     : launch_pdl(pool_kernel<false>, grid, block, 0, s, a, 1);
+  }
   const int E = a.T / a.m;
-  if (E == 0 || (a.entries == nullptr && a.fp4 == nullptr)) return cudaSuccess;
+  if (E == 0) return cudaSuccess;
   const int epc = a.m >= 32 ? 1 : (a.m >= 8 ? 4 : 16);
   const dim3 grid((E + epc - 1) / epc, a.B), block(a.C / 2);
   return a.in_bf16 ? launch_pdl(pool_kernel<true>, grid, block, 0, s, a, epc)

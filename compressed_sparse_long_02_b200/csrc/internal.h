@@ -96,6 +96,11 @@ struct PoolArgs {
   int E_max;
   uint8_t* fp4;       // nullable, [B, E_max, C/2]
   uint8_t* fp4_scale; // nullable, [B, E_max, C/32]
+  // Streaming (decode) mode when non-null: device [B], the position of each sequence's
+  // newest token; kv / logits are then [B, (1+overlap)*m, C], row s holding token
+  // pos - (1+overlap)*m + 1 + s, and only the entry that token completes is written.
+  const int32_t* pos;
+  int32_t* err;       // device error word (streaming mode: an entry index past E_max)
 };
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
 

@@ -9,6 +9,7 @@
  *   csa_compress        every m tokens -> one KV entry by per-channel softmax pooling
  *                       (CSA: m = 4, each entry also pools the previous group of 4;
  *                       HCA: m' = 128, no overlap), then RMSNorm and partial RoPE.
+ *   csa_compress_step   the same for decode: the entry a new token completes.
  *   csa_norm_rope       RMSNorm + partial RoPE of query heads (and raw window rows).
  *   csa_quantize_mxfp4  FP4 (E2M1, UE8M0 scale per 32) encoding for the lightning indexer.
  *   csa_index_topk      lightning-indexer scores of every visible entry, then top-k.
@@ -113,6 +114,27 @@ typedef struct {
 CSA_API csa_status csa_compress(const csa_pool_cfg* cfg, int B, int T, const void* kv, const void* logits,
                         const float* slot_bias, void* entries, int E_max, uint8_t* fp4_out,
                         uint8_t* fp4_scale, void* window_kv, cudaStream_t stream);
+
+/*
+ * csa_compress_step -- the compressor during decode (a token at a time): for each
+ * sequence b whose newest token, at position pos[b], completes a group
+ * ((pos[b] + 1) % m == 0), entry j = (pos[b] + 1) / m - 1 exactly as csa_compress
+ * writes it for the whole sequence (same pooling, norm, RoPE at position pos[b] and
+ * MXFP4 key), computed from the sequence's last S = (1 + overlap) * m raw tokens.
+ * ("DeepSeek-V4: Million-Token Context": at decode a new entry appears every m-th
+ * token; the window covers the tokens of the unfinished group.)
+ *
+ * pos: device int32 [B].  kv, logits: [B, S, C] (cfg->in_dtype), row s holding token
+ * pos[b] - S + 1 + s (rows of tokens before position 0 are ignored: entry 0 pools its
+ * own group only).  entries / fp4_out / fp4_scale as in csa_compress.  Nothing is
+ * written for a sequence whose group is incomplete; an entry index j >= E_max is
+ * skipped and flags CSA_DEVERR_INDEX.  The new token's window row is
+ * csa_norm_rope of kv at pos[b].
+ * Errors: as csa_compress; INVALID_ARG for B < 0, E_max < 1 or a NULL pos / kv / logits.
+ */
+CSA_API csa_status csa_compress_step(const csa_pool_cfg* cfg, int B, const int32_t* pos, const void* kv,
+                                     const void* logits, const float* slot_bias, void* entries, int E_max,
+                                     uint8_t* fp4_out, uint8_t* fp4_scale, cudaStream_t stream);
 
 /*
  * csa_norm_rope -- RMSNorm (unit gain) and partial RoPE of `heads` vectors per row
