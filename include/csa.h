@@ -121,8 +121,10 @@ CSA_API csa_status csa_compress(const csa_pool_cfg* cfg, int B, int T, const voi
  * ((pos[b] + 1) % m == 0), entry j = (pos[b] + 1) / m - 1 exactly as csa_compress
  * writes it for the whole sequence (same pooling, norm, RoPE at position pos[b] and
  * MXFP4 key), computed from the sequence's last S = (1 + overlap) * m raw tokens.
- * ("DeepSeek-V4: Million-Token Context": at decode a new entry appears every m-th
- * token; the window covers the tokens of the unfinished group.)
+ * ("Follow the white rabbit: DeepSeek V4's architecture in 3D", sliding-window
+ * paragraph: a group becomes a compressed entry once it is complete, and the tokens of
+ * the unfinished group reach attention through the window; so at decode a new entry
+ * appears every m-th token.)
  *
  * pos: device int32 [B].  kv, logits: [B, S, C] (cfg->in_dtype), row s holding token
  * pos[b] - S + 1 + s (rows of tokens before position 0 are ignored: entry 0 pools its
