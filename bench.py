@@ -54,7 +54,7 @@ def load_peaks() -> dict:
 # at capture time: a kernel changed since its capture reports traffic null.
 NCU_TRAFFIC = {
     "attention": {"bytes": 40084736 + 724480, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
-                  "sha1": "f897a6bd6b9c4b5200347d0c2b4becef86f2bcaf"},
+                  "sha1": "eaa29fa8aad8865cf064ea5c1fbdfbb6548616c8"},
     "index_score": {"bytes": 71479552 + 1724928, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
                     "sha1": "92645beee700a6035b78e2d12283f92df90069dd"},
     "topk_select": {"bytes": 4252672, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",

@@ -18,7 +18,7 @@ import torch
 __all__ = ["CsaError", "lib", "csa_compress", "csa_compress_step", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk",
            "csa_index_score", "csa_index_score_q", "csa_topk_select",
            "csa_index_topk_workspace", "csa_sparse_attn", "csa_sparse_attn_workspace", "hca_attn",
-           "hca_attn_workspace", "csa_get_device_error", "LIB_PATH", "DEVERR_NONE", "DEVERR_TIMEOUT",
+           "hca_attn_workspace", "csa_get_device_error", "csa_set_batch_invariant", "LIB_PATH", "DEVERR_NONE", "DEVERR_TIMEOUT",
            "DEVERR_INDEX"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcsa.so")
@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
             L.hca_attn_workspace.argtypes = [I, I, I, I, I]
             L.hca_attn_workspace.restype = SZ
             L.csa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
+            L.csa_set_batch_invariant.argtypes = [I]
+            L.csa_set_batch_invariant.restype = I
             L.csa_status_string.argtypes = [I]
             L.csa_status_string.restype = ctypes.c_char_p
             L.csa_last_cuda_error.argtypes = []
@@ -318,6 +320,11 @@ def hca_attn(q, q_pos, q_seq, entries, n_entries, window, window_base, *, mprime
                         _ptr(workspace), workspace.numel(), _stream(q))
     _check("hca_attn", st)
     return out, lse
+
+
+def csa_set_batch_invariant(on: bool) -> None:
+    """Process-wide: attention splits each query's keys by a rule independent of the batch."""
+    _check("csa_set_batch_invariant", lib().csa_set_batch_invariant(int(bool(on))))
 
 
 def csa_get_device_error(device=None) -> int:

@@ -70,6 +70,11 @@ const char* csa_last_cuda_error(void) {
   return buf;
 }
 
+csa_status csa_set_batch_invariant(int on) {
+  set_batch_invariant(on != 0);
+  return CSA_OK;
+}
+
 const char* csa_status_string(csa_status s) {
   switch (s) {
     case CSA_OK: return "ok";

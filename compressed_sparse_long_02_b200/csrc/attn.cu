@@ -35,6 +35,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 
@@ -771,9 +772,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
 
 int g_attn_smem[64];
 
+std::atomic<int> g_batch_invariant{0};
+
+}  // namespace
+
+void set_batch_invariant(bool on) { g_batch_invariant.store(on ? 1 : 0); }
+bool batch_invariant() { return g_batch_invariant.load() != 0; }
+
+namespace {
+
 // Splits of one query's key list: a power of two up to the portable cluster size, so
-// that the CTAs of a query fill about one wave of SMs.
+// that the CTAs of a query fill about one wave of SMs.  In batch-invariant mode the
+// count depends on the key count alone, so a query's split boundaries, partials and
+// merge order (and with them every output bit) do not depend on the batch it is in.
 int split_count(int Nq, int max_keys) {
+  if (batch_invariant()) {  // the fewest power-of-two splits of at most 512 rows each, up to 8
+    int s = 1;
+    while (s < kMaxSplits && static_cast<int64_t>(s) * 512 < max_keys) s *= 2;
+    return s;
+  }
   const int tiles = std::max(1, (max_keys + kBN - 1) / kBN);
   if (Nq >= kSplitSMs) return 1;
   const int want = std::min(tiles, kSplitSMs / std::max(1, Nq));

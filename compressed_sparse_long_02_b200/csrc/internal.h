@@ -158,6 +158,10 @@ struct AttnArgs {
   size_t ws_bytes;
 };
 size_t attn_workspace_bytes(int Nq, int H, int D, int max_keys);
+// Batch-invariant attention (process-wide, off by default): a query's key list is split
+// by a rule that depends on the key count only, never on the batch.
+void set_batch_invariant(bool on);
+bool batch_invariant();
 cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s);
 
 }  // namespace csa

@@ -284,6 +284,19 @@ CSA_API size_t hca_attn_workspace(int Nq, int H, int D, int E_max, int W);
  * *code_out and clears it.  CSA_ERR_CUDA if the stream reports an error. */
 CSA_API csa_status csa_get_device_error(int32_t* code_out, cudaStream_t stream);
 
+/*
+ * csa_set_batch_invariant -- process-wide switch (off by default) for batch-invariant
+ * results.  With it on, csa_sparse_attn and hca_attn split each query's key list into
+ * the fewest power-of-two parts of at most 512 rows (at most 8 parts), a rule that
+ * depends on k + W (or E_max + W) only.  A query's output is then bitwise the same
+ * whatever batch it is computed in, and the decode calls reproduce the prefill's
+ * outputs bit for bit.  Every other call is batch-invariant already: indexer scores
+ * are a fixed per-pair chain, top-k is exact, and csa_compress_step writes
+ * csa_compress's entries.  The workspace sizes follow the setting: query them after
+ * setting it.
+ */
+CSA_API csa_status csa_set_batch_invariant(int on);
+
 /* Static description of a status code. */
 CSA_API const char* csa_status_string(csa_status status);
 
