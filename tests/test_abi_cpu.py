@@ -75,3 +75,26 @@ def test_workspace_sizes(L):
     assert B.csa_sparse_attn_workspace(8192, 64, 512, 512, 128) <= 256
     # decode: split partials of fp32 [splits, 64, 512] per query
     assert B.csa_sparse_attn_workspace(32, 64, 512, 1024, 128) >= 32 * 2 * 64 * 512 * 4
+
+
+def test_batch_invariant_split_rule(L):
+    """With the batch-invariant switch on, the attention split of a query depends on
+    k + W only: the workspace per query (its partials) is the same for every batch size,
+    the fewest power-of-two splits of at most 512 rows (at most 8).  Off, few queries are
+    split more ways than many."""
+    from compressed_sparse_long_02_b200 import binding as B
+
+    def per_query_splits(Nq, k, W):
+        ws = B.csa_sparse_attn_workspace(Nq, 64, 512, k, W)
+        return 0 if ws <= 256 else round((ws - 512) / (Nq * 64 * (512 * 4 + 8)))
+
+    try:
+        B.csa_set_batch_invariant(True)
+        for k, W, want in [(64, 128, 0), (448, 64, 0), (512, 128, 2), (1024, 128, 4), (2048, 128, 8),
+                           (262144, 128, 8)]:
+            got = {per_query_splits(Nq, k, W) for Nq in (1, 3, 32, 148, 8192)}
+            assert got == {want}, f"k={k}, W={W}: splits {got}, expected {want} for every batch"
+    finally:
+        B.csa_set_batch_invariant(False)
+    assert per_query_splits(1, 1024, 128) == 8 and per_query_splits(32, 1024, 128) == 4
+    assert per_query_splits(8192, 1024, 128) == 0
