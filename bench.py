@@ -58,7 +58,7 @@ NCU_TRAFFIC = {
     "index_score": {"bytes": 71479552 + 1724928, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
                     "sha1": "92645beee700a6035b78e2d12283f92df90069dd"},
     "topk_select": {"bytes": 4252672, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",
-                    "sha1": "58b7e4b5c9975a744f5b58160cfdafb4cf85ff3c"},
+                    "sha1": "a2d57f7f3c5bef183b3959e4a1cf4ac3611c4eaa"},
 }
 
 
