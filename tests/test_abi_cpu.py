@@ -53,6 +53,15 @@ def test_validation_without_device(L):
     assert L.csa_compress(ctypes.byref(cfg), 1, 8, P(16), P(16), P(16), None, 2, None, None, None, None) == 1
     cfg = B._PoolCfg(4, 1, 128, 0, 1e-6, 0, 1e4, 0)  # misaligned input pointer
     assert L.csa_compress(ctypes.byref(cfg), 1, 8, P(17), P(16), P(16), None, 2, None, None, None, None) == 2
+    # decode-time compressor: no positions, misaligned rows, unsupported channels, nothing to do
+    L.csa_compress_step.argtypes = [ctypes.POINTER(B._PoolCfg), ctypes.c_int, P, P, P, P, P, ctypes.c_int, P, P, P]
+    cfg = B._PoolCfg(4, 1, 128, 0, 1e-6, 0, 1e4, 0)
+    assert L.csa_compress_step(ctypes.byref(cfg), 2, None, P(16), P(16), P(16), P(16), 8, None, None, None) == 1
+    assert L.csa_compress_step(ctypes.byref(cfg), 2, P(16), P(24), P(16), P(16), P(16), 8, None, None, None) == 2
+    assert L.csa_compress_step(ctypes.byref(cfg), 2, P(16), P(16), P(16), P(16), P(16), 0, None, None, None) == 1
+    assert L.csa_compress_step(ctypes.byref(cfg), 0, None, None, None, None, None, 8, None, None, None) == 0
+    cfg = B._PoolCfg(4, 1, 96, 0, 1e-6, 0, 1e4, 0)
+    assert L.csa_compress_step(ctypes.byref(cfg), 2, P(16), P(16), P(16), P(16), P(16), 8, None, None, None) == 3
     # quantiser: cols not a multiple of 32
     assert L.csa_quantize_mxfp4(P(16), 0, 4, 48, P(16), P(16), None) == 1
     # indexer: unsupported head dim, E_max not a multiple of 8, workspace too small
