@@ -56,7 +56,7 @@ NCU_TRAFFIC = {
     "attention": {"bytes": 40084736 + 724480, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
                   "sha1": "eaa29fa8aad8865cf064ea5c1fbdfbb6548616c8"},
     "index_score": {"bytes": 71479552 + 1724928, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
-                    "sha1": "92645beee700a6035b78e2d12283f92df90069dd"},
+                    "sha1": "765ad86bbe490ed1a125c7e5bff8b126b3b9a484"},
     "topk_select": {"bytes": 4252672, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",
                     "sha1": "a2d57f7f3c5bef183b3959e4a1cf4ac3611c4eaa"},
 }

@@ -375,7 +375,12 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
 //                head-weighted fp32 chain, store
 // A block whose queries span several sequences runs as segments, one per sequence run,
 // each with its own key tiles; the pairs a segment touches compute both halves and keep
-// the segment's queries.  Every role derives the same (segment, tile, pair) order.
+// the segment's queries.  The producer writes each block's query information (validity,
+// visible counts, segments) into shared memory beside the block buffer, published by the
+// buffer's barrier, so every role follows the same (segment, tile, pair) order; a block
+// without a valid query still passes through the buffer protocol.  Every wait sleeps
+// (try_wait with a suspend-time hint) instead of polling: 26 warps polling mbarriers
+// took shared-memory bandwidth from the warps doing the work.
 constexpr int kPStages = 10;
 constexpr int kBlkQ = 8;               // queries per block
 constexpr int kPairs = kBlkQ / 2;      // N = 128 MMAs per key tile
