@@ -24,13 +24,17 @@ bool pow2_channels(int C) { return C == 64 || C == 128 || C == 256 || C == 512 |
 
 thread_local cudaError_t g_last_cuda = cudaSuccess;
 
-csa_status from_cuda(cudaError_t e) {
+}  // namespace
+
+csa_status status_from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return CSA_OK;
   if (e == cudaErrorInvalidValue) return CSA_ERR_INVALID_ARG;
   g_last_cuda = e;
   return CSA_ERR_CUDA;
 }
 
+namespace {
+csa_status from_cuda(cudaError_t e) { return status_from_cuda(e); }
 }  // namespace
 
 int32_t* device_error_word() {

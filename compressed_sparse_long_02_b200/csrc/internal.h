@@ -12,6 +12,9 @@ namespace csa {
 
 // device error word of the current device (lazily resolved, cached per device)
 int32_t* device_error_word();
+// Status of a CUDA result; a failure other than cudaErrorInvalidValue is remembered as
+// the calling thread's last CUDA error (csa_last_cuda_error) and gives CSA_ERR_CUDA.
+csa_status status_from_cuda(cudaError_t e);
 int num_sms();
 
 // Raise `fn`'s dynamic shared-memory limit to `bytes` on the current device (once per

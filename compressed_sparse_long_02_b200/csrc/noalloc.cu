@@ -32,17 +32,24 @@ constexpr int kMaxDevices = 64;
 float* g_static_scores_addr[kMaxDevices];
 std::mutex g_static_mu;
 
-// device address of g_static_scores on the current device (resolved on first use)
-float* static_scores() {
+// Device address of g_static_scores on the current device (resolved on first use) in
+// *out; the CUDA result of the lookup (a failure is reported like a failed launch).
+cudaError_t static_scores(float** out) {
+  *out = nullptr;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lk(g_static_mu);
   if (g_static_scores_addr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scores) != cudaSuccess || p == nullptr) return nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scores);
+    if (e != cudaSuccess) return e;
+    if (p == nullptr) return cudaErrorInvalidSymbol;
     g_static_scores_addr[dev] = static_cast<float*>(p);
   }
-  return g_static_scores_addr[dev];
+  *out = g_static_scores_addr[dev];
+  return cudaSuccess;
 }
 
 bool is_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -65,8 +72,9 @@ extern "C" csa_status csa_index_topk_static(int Nq, int Hi, int Di, int k, int m
   if (!q_fp4 || !q_scale || !w || !q_pos || !q_seq || !k_fp4 || !k_scale || !n_entries || !idx_out || !cnt_out)
     return CSA_ERR_INVALID_ARG;
   if (!is_aligned16(q_fp4) || !is_aligned16(k_fp4) || !is_aligned16(k_scale)) return CSA_ERR_ALIGNMENT;
-  float* scratch = static_scores();
-  if (scratch == nullptr) return CSA_ERR_CUDA;
+  float* scratch = nullptr;
+  const cudaError_t se = static_scores(&scratch);
+  if (se != cudaSuccess) return status_from_cuda(se == cudaErrorInvalidValue ? cudaErrorInvalidSymbol : se);
   IndexArgs a{};
   a.Nq = Nq;
   a.Hi = Hi;
@@ -88,7 +96,5 @@ extern "C" csa_status csa_index_topk_static(int Nq, int Hi, int Di, int k, int m
   a.score_out = nullptr;
   a.scores_ws = scratch;
   a.E_stride = E_stride;
-  const cudaError_t e = launch_index_topk(a, stream);
-  if (e == cudaSuccess) return CSA_OK;
-  return e == cudaErrorInvalidValue ? CSA_ERR_INVALID_ARG : CSA_ERR_CUDA;
+  return status_from_cuda(launch_index_topk(a, stream));
 }

@@ -18,8 +18,10 @@
  *
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers unless marked "host".  The caller
- *     owns every buffer; the library allocates nothing on these calls and keeps
- *     only one lazily created 4-byte device error word per device.
+ *     owns every buffer; the library allocates nothing on these calls.  It keeps a
+ *     4-byte device error word per device and, on every device that loads its
+ *     module, the fixed 8 MiB scratch array of csa_index_topk_static (resident
+ *     whether or not that call is ever made).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream).  Only argument validation is synchronous.  Results are ready when
  *     the stream reaches the call.
@@ -296,6 +298,32 @@ CSA_API csa_status csa_get_device_error(int32_t* code_out, cudaStream_t stream);
  * setting it.
  */
 CSA_API csa_status csa_set_batch_invariant(int on);
+
+/*
+ * csa_selftest_bounded_wait -- exercises the failure-detection path of the pipelines:
+ * every wait of a kernel in this library on a pipeline barrier gives up after a bounded
+ * number of SM cycles (about 2 s), records CSA_DEVERR_TIMEOUT in the device error word
+ * and releases the kernel's other roles through a shared abort flag, so a lost arrival
+ * ends the kernel instead of hanging the GPU.  This launches one CTA whose two warps wait
+ * on barriers that nothing ever completes (sleeping = 1: the suspend-hinted wait of the
+ * many-warp roles; 0: the polling wait); warp 1 starts a quarter of the limit later.
+ * out (device int64 [4]): per warp, 1 if its wait succeeded (never, here) else 0, then
+ * the SM cycles it waited.  Afterwards csa_get_device_error reports CSA_DEVERR_TIMEOUT;
+ * the context stays usable.  The pages have no counterpart: this is a test hook.
+ */
+CSA_API csa_status csa_selftest_bounded_wait(int sleeping, long long* out, cudaStream_t stream);
+
+/*
+ * csa_mma_peak_probe -- dense tensor-core throughput probe (a measurement aid; the pages
+ * have no counterpart).  `ctas` CTAs (one per SM) each issue `iters` rounds of four
+ * tcgen05 MMAs of M = 128, N (16..256, a multiple of 16) and K = 64 block-scaled FP4
+ * elements (mxf4 = 1, kind::mxf4.block_scale) or K = 16 bf16 elements (mxf4 = 0,
+ * kind::f16) on operands resident in shared memory, so no memory traffic limits the
+ * rate.  *flops_out (host, may be NULL) receives the launch's dense FLOPs (2 M N K per
+ * MMA); time the call with events on `stream`.  Operand values are a fixed pattern
+ * and the output is discarded.
+ */
+CSA_API csa_status csa_mma_peak_probe(int mxf4, int N, int iters, int ctas, double* flops_out, cudaStream_t stream);
 
 /* Static description of a status code. */
 CSA_API const char* csa_status_string(csa_status status);

@@ -97,3 +97,49 @@ def fp4_mismatch_justified(x_ref: np.ndarray, packed_gpu: np.ndarray, scales_gpu
     code_bad = cg != cr
     assert not (code_bad & ~near & ~blk_edge).any(), "E2M1 code differs away from a rounding boundary"
     return int(code_bad.sum() + sc_bad.sum())
+
+
+def check_csa_prefill_rows(wl, host: dict, r: dict, rows: np.ndarray, check_entries: bool = True) -> dict:
+    """Per-row parity of one CSA prefill layer run against the oracle.
+
+    host: host arrays of one sequence's inputs (kv, z, bias, ki, zi, bias_i: full length;
+    q, qi, w: only the query rows `rows`, in that order).  r: the layer's device outputs
+    for every token as a query (entries, k_fp4, k_scale, q_fp4, q_scale, idx, cnt, out).
+
+    Every sampled row must pass, none is allowed to miss:
+    * the GPU pools indexer keys in float32 and the oracle in float64, so a key's MXFP4
+      code may differ only where the float64 value sits on a rounding or scale boundary
+      (`fp4_mismatch_justified`);
+    * the query bytes are a pure function of the input bits: equal;
+    * the oracle's scores and top-k over the GPU's key bytes: the GPU's index set equals
+      the oracle's on every row, up to the 1e-6 tie exemption (`check_topk`);
+    * the oracle's attention over that index set: within the attention tolerance.
+    Returns counts (justified FP4 differences, exempt rows)."""
+    import oracle
+    E = wl.T // wl.m
+    seq = np.zeros(len(rows), np.int32)
+    ki_ref = oracle.pool(host["ki"], host["zi"], host["bias_i"], wl.m, wl.overlap)
+    kp_ref, ks_ref = oracle.mxfp4_quantize(ki_ref.astype(np.float32))
+    kp_gpu = t2np(r["k_fp4"])[0, :E]
+    ks_gpu = t2np(r["k_scale"])[0, :E]
+    n_fp4 = fp4_mismatch_justified(ki_ref, kp_gpu, ks_gpu, kp_ref, ks_ref)
+    qi = host["qi"]
+    qi = bf16_bits_to_f64(qi).astype(np.float32) if qi.dtype == np.uint16 else qi.astype(np.float32)
+    qp, qs = oracle.mxfp4_quantize(qi)
+    sel = np.asarray(rows)
+    assert np.array_equal(t2np(r["q_fp4"])[sel], qp) and np.array_equal(t2np(r["q_scale"])[sel], qs), \
+        "indexer query bytes differ"
+    n_vis = np.array([oracle.n_visible(t, wl.m, E) for t in rows], np.int32)
+    s32, _, _ = oracle.index_scores(qp, qs, host["w"], seq, n_vis, kp_gpu[None], ks_gpu[None])
+    idx_ref, cnt_ref, kth = oracle.topk(s32, n_vis, wl.k)
+    idx_gpu, cnt_gpu = t2np(r["idx"])[sel], t2np(r["cnt"])[sel]
+    exempt = check_topk(idx_gpu, cnt_gpu, idx_ref, cnt_ref, kth, s32, n_vis, wl.k)
+    ent = oracle.entries_rows(host["kv"], host["z"], host["bias"], wl.m, wl.overlap, wl.norm, wl.eps, wl.rope_dims,
+                              wl.theta)
+    if check_entries:
+        assert_bf16_rounding(t2np(r["entries"])[0, :E], ent, "entries")
+    win = oracle.window_rows(host["kv"], wl.norm, wl.eps, wl.rope_dims, wl.theta)
+    qf = oracle.prep_queries(host["q"], rows, wl.norm, wl.eps, wl.rope_dims, wl.theta)
+    out_ref, _ = oracle.attention(qf, rows, seq, ent[None], idx_gpu, cnt_gpu, win[None], np.zeros(1, np.int64), wl.W)
+    assert_close_attn(t2np(r["out"])[sel], out_ref, f"CSA prefill T={wl.T}")
+    return {"fp4_justified": n_fp4, "exempt_rows": exempt}

@@ -107,3 +107,22 @@ def test_batch_invariant_split_rule(L):
         B.csa_set_batch_invariant(False)
     assert per_query_splits(1, 1024, 128) == 8 and per_query_splits(32, 1024, 128) == 4
     assert per_query_splits(8192, 1024, 128) == 0
+
+
+def test_static_indexer_size_limit_boundary(L):
+    """csa_index_topk_static holds Nq * round_up(E_max, 4) <= 2^21 scores.  The size check runs
+    before any device work, so null pointers reach it: a call exactly at the limit passes it
+    (and then stops at the null pointers), one row of 8 entries more is rejected as too large
+    for the scratch, and E_max not a multiple of 8 is unsupported."""
+    P, I = ctypes.c_void_p, ctypes.c_int
+    L.csa_index_topk_static.argtypes = [I, I, I, I, I, P, P, P, P, P, I, I, P, P, P, P, P, P]
+    L.csa_index_topk_static.restype = I
+
+    def call(Nq, E_max):
+        return L.csa_index_topk_static(Nq, 64, 128, 8, 4, *([None] * 5), 1, E_max, *([None] * 5), None)
+
+    assert call(32, 65536) == 1          # 32 x 65536 = 2^21: within the limit, then INVALID_ARG
+    assert call(32, 65544) == 4          # one more multiple of 8: CSA_ERR_WORKSPACE
+    assert call(1, 1 << 21) == 1
+    assert call(1, (1 << 21) + 8) == 4
+    assert call(32, 65540) == 3          # E_max % 8 != 0: CSA_ERR_UNSUPPORTED

@@ -6,7 +6,10 @@ exactly the entry `csa_compress` writes for the whole sequence: the same pooling
 RMSNorm, RoPE and MXFP4 key, bit for bit (the two run the same arithmetic in the same
 order; `csa_compress` itself is checked against the oracle in test_gpu_kernels.py).
 Rows of tokens before position 0 must be ignored, sequences whose group is incomplete
-must be left alone, and an entry index past E_max must be skipped and flagged.
+must be left alone, and an entry index past E_max must be skipped and flagged.  The
+entries it writes are also checked against the oracle directly: bf16 values within one
+bf16 rounding of the float64 pooling, norm and RoPE, and MXFP4 keys equal to the oracle's
+encoding except where a float64 value sits on a rounding or scale boundary.
 """
 import numpy as np
 import pytest
@@ -14,7 +17,7 @@ import torch
 
 import oracle
 from compressed_sparse_long_02_b200 import synth
-from tests.helpers import assert_close_attn, t2np, to_dev, to_dev_bf16
+from tests.helpers import assert_bf16_rounding, assert_close_attn, fp4_mismatch_justified, t2np, to_dev, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +60,11 @@ def test_compress_step_matches_whole_sequence(B, cuda, name, T):
             if lo + s >= 0:
                 ring_kv[b, s] = kv_t[lo + s]
                 ring_z[b, s] = z_t[lo + s]
+    # the oracle's entries and MXFP4 keys of the same sequence (pooled before norm / RoPE)
+    ent_ref = oracle.entries_rows(inp["kv"][0], inp["z"][0], inp["bias"], m, wl.overlap, wl.norm, wl.eps,
+                                  wl.rope_dims, wl.theta)
+    pool_ref = oracle.pool(inp["kv"][0], inp["z"][0], inp["bias"], m, wl.overlap)
+    kp_ref, ks_ref = oracle.mxfp4_quantize(pool_ref.astype(np.float32))
     sentinel = 0x4444
     ent = torch.full((Bs, E, wl.C), sentinel, dtype=torch.int16, device=cuda)
     fp4 = torch.full((Bs, E, wl.C // 2), 0x55, dtype=torch.uint8, device=cuda)
@@ -70,6 +78,10 @@ def test_compress_step_matches_whole_sequence(B, cuda, name, T):
             j = (p + 1) // m - 1
             assert torch.equal(ent[b, j], ent_full[j]), f"{name}: entry {j} differs from the whole-sequence one"
             assert torch.equal(fp4[b, j], fp4_full[j]) and torch.equal(sc[b, j], sc_full[j]), f"{name}: fp4 key {j}"
+            got = t2np(ent[b, j].view(torch.bfloat16))[None]
+            assert_bf16_rounding(got, ent_ref[j][None], f"{name}: entry {j} vs the oracle")
+            fp4_mismatch_justified(pool_ref[j][None], t2np(fp4[b, j])[None], t2np(sc[b, j])[None], kp_ref[j][None],
+                                   ks_ref[j][None])
             rows[j] = False
         assert bool((ent[b][rows] == sentinel).all()), f"{name}: row {b} wrote outside its entry"
         assert bool((fp4[b][rows] == 0x55).all()) and bool((sc[b][rows] == 0x66).all())
