@@ -28,7 +28,7 @@ import math
 import numpy as np
 
 __all__ = ["Workload", "WORKLOADS", "prefill_inputs", "prefill_inputs_torch", "decode_inputs",
-           "decode_inputs_torch", "to_dtype_np"]
+           "decode_inputs_torch", "to_dtype_np", "ProjShape", "PROJ", "proj_inputs", "proj_inputs_torch"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -218,3 +218,48 @@ def decode_inputs_torch(wl: Workload, device, B: int | None = None, E: int | Non
         "window": torch.randn((B, W, D), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16),
         "pos": torch.full((B,), E * wl.m - 1, dtype=torch.int32, device=device),
     }
+
+
+# ----------------------------------------------------------------------------- output projection
+@dataclasses.dataclass(frozen=True)
+class ProjShape:
+    """Grouped output projection after core attention (the pages name it, "DeepSeek-V4:
+    Towards Highly Efficient ..." section 2.3, without sizes): H heads of D in G groups,
+    R values per group, then d_model.  R and d_model are synthetic choices."""
+    T: int
+    H: int = 64
+    D: int = 512
+    G: int = 8
+    R: int = 1024
+    d_model: int = 4096
+    seed: int = 6
+
+
+PROJ = {"tiny": ProjShape(T=37, H=16, D=128, G=4, R=256, d_model=512),
+        "csa_prefill_8k": ProjShape(T=8192)}
+
+
+def proj_inputs(ps: ProjShape, T: int | None = None) -> dict:
+    """Host inputs (bf16 bits): o [T, H, D] ~ N(0,1); A [G, R, (H/G) D] ~ N(0, 1/((H/G) D));
+    Bm [d_model, G R] ~ N(0, 1/(G R)), so the intermediate and the output are ~N(0,1)."""
+    T = ps.T if T is None else T
+    rng = np.random.default_rng(ps.seed)
+    Kg = (ps.H // ps.G) * ps.D
+    return {"o": to_dtype_np(_normal(rng, (T, ps.H, ps.D)), "bf16"),
+            "A": to_dtype_np(_normal(rng, (ps.G, ps.R, Kg), 1.0 / Kg), "bf16"),
+            "Bm": to_dtype_np(_normal(rng, (ps.d_model, ps.G * ps.R), 1.0 / (ps.G * ps.R)), "bf16")}
+
+
+def proj_inputs_torch(ps: ProjShape, device, T: int | None = None) -> dict:
+    """The same shapes and distributions drawn on ``device`` (bf16 tensors)."""
+    import torch
+    T = ps.T if T is None else T
+    g = torch.Generator(device=device)
+    g.manual_seed(ps.seed * 7919 + 31)
+    Kg = (ps.H // ps.G) * ps.D
+
+    def nrm(shape, var=1.0):
+        return (torch.randn(shape, generator=g, device=device) * math.sqrt(var)).to(torch.bfloat16)
+
+    return {"o": nrm((T, ps.H, ps.D)), "A": nrm((ps.G, ps.R, Kg), 1.0 / Kg),
+            "Bm": nrm((ps.d_model, ps.G * ps.R), 1.0 / (ps.G * ps.R))}

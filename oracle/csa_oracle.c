@@ -299,3 +299,28 @@ void orc_attention(int nq, int H, int D, double scale, int q_dt, const void* q, 
     free(row_src);
   }
 }
+
+void orc_grouped_out_proj(int T, int H, int D, int G, int R, int d_model, int in_dt, const void* o, const void* A,
+                          const void* Bm, double* z, double* y) {
+  const int64_t Kg = (int64_t)(H / G) * D;  /* inputs per group */
+  const int64_t HD = (int64_t)H * D;
+  const int64_t GR = (int64_t)G * R;
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < T; ++t) {
+    /* each group: its heads' outputs times the group's own matrix */
+    for (int g = 0; g < G; ++g) {
+      for (int r = 0; r < R; ++r) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < Kg; ++i)
+          acc += ld_elem(o, in_dt, (int64_t)t * HD + g * Kg + i) * ld_elem(A, in_dt, ((int64_t)g * R + r) * Kg + i);
+        z[(int64_t)t * GR + (int64_t)g * R + r] = acc;
+      }
+    }
+    /* the groups' results, concatenated, times the dense matrix */
+    for (int n = 0; n < d_model; ++n) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < GR; ++j) acc += z[(int64_t)t * GR + j] * ld_elem(Bm, in_dt, (int64_t)n * GR + j);
+      y[(int64_t)t * d_model + n] = acc;
+    }
+  }
+}

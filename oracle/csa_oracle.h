@@ -112,6 +112,20 @@ void orc_attention(int nq, int H, int D, double scale, int q_dt, const void* q, 
                    const int32_t* idx, const int32_t* cnt, int W, int Tw, int w_dt, const void* window,
                    const int64_t* wbase, double* out, double* lse);
 
+/* Grouped output projection ([SUMM] 2.3, "Shared KV and output projection": after core
+ * attention, a grouped projection carries the many head outputs back to the hidden state
+ * at less cost than one dense projection).  The pages name the grouping but no sizes or
+ * structure; the reading taken: the H heads form G groups of H/G consecutive heads; each
+ * group's concatenated outputs (H/G * D values) are projected by the group's own matrix
+ * to R values; the G * R values are then projected by one dense matrix to d_model:
+ *   z[t, g*R + r] = sum_{i < (H/G)*D} o[t, g*(H/G)*D + i] * A[g, r, i]
+ *   y[t, n]       = sum_{j < G*R} z[t, j] * Bm[n, j]
+ * o [T, H*D], A [G, R, (H/G)*D], Bm [d_model, G*R] (element type in_dt each);
+ * z [T, G*R] and y [T, d_model] double.  y is computed from the double z (no rounding
+ * of the intermediate).  H must be a multiple of G. */
+void orc_grouped_out_proj(int T, int H, int D, int G, int R, int d_model, int in_dt, const void* o, const void* A,
+                          const void* Bm, double* z, double* y);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,7 @@ import numpy as np
 __all__ = [
     "build", "lib", "n_visible", "pool", "rmsnorm", "rope", "mxfp4_quantize", "mxfp4_dequantize",
     "index_scores", "topk", "attention", "hca_select", "csa_prefill", "hca_prefill", "csa_decode",
-    "window_rows", "prep_queries", "entries_rows", "F64", "F32", "BF16",
+    "window_rows", "prep_queries", "entries_rows", "grouped_out_proj", "F64", "F32", "BF16",
 ]
 
 F64, F32, BF16 = 0, 1, 2
@@ -61,6 +61,7 @@ def lib():
             L.orc_index_scores.restype = I64
             L.orc_topk.argtypes = [I, I, P, P, I, P, P, P]
             L.orc_attention.argtypes = [I, I, I, D, I, P, P, P, I, I, P, I, P, P, I, I, I, P, P, P, P]
+            L.orc_grouped_out_proj.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P]
             _lib = L
     return _lib
 
@@ -289,3 +290,24 @@ def csa_decode(wl, entries, k_packed, k_scales, q, qi_packed, qi_scales, w, wind
     out, lse = attention(q[seqs], np.asarray(pos)[seqs], seqs.astype(np.int32), entries, idx, cnt, window,
                          wbase, wl.W)
     return dict(scores=s32, n_vis=n_vis, idx=idx, cnt=cnt, kth=kth, out=out, lse=lse, inexact=bad)
+
+
+def grouped_out_proj(o, A, Bm, G: int):
+    """Grouped output projection: o [T, H, D] (or [T, H*D]); A [G, R, (H/G)*D]; Bm [d_model, G*R];
+    all of one element type (float64, float32 or bf16 bits).  Returns (z [T, G*R], y [T, d_model])
+    in float64."""
+    o, A, Bm = _c(o), _c(A), _c(Bm)
+    assert o.dtype == A.dtype == Bm.dtype
+    T = o.shape[0]
+    HD = int(np.prod(o.shape[1:]))
+    Gc, R, Kg = A.shape
+    assert Gc == G and Kg * G == HD
+    d_model, GR = Bm.shape
+    assert GR == G * R
+    # heads and head dim only enter through their product and the group split
+    H, D = (o.shape[1], o.shape[2]) if o.ndim == 3 else (G, Kg)
+    assert H % G == 0 and (H // G) * D == Kg
+    z = np.zeros((T, G * R), dtype=np.float64)
+    y = np.zeros((T, d_model), dtype=np.float64)
+    lib().orc_grouped_out_proj(T, H, D, G, R, d_model, _dt(o), _p(o), _p(A), _p(Bm), _p(z), _p(y))
+    return z, y

@@ -399,3 +399,64 @@ def test_tiny_workload_sanity():
     t = np.arange(512)
     np.testing.assert_array_equal(r["cnt"], np.minimum((t + 1) // 4, wl.k))
     assert np.all(np.isfinite(r["out"]))
+
+
+# ------------------------------------------------------------------ grouped output projection
+def _gop_case(seed, T=5, H=8, D=6, G=4, R=5, dm=7):
+    rng = np.random.default_rng(seed)
+    o = rng.standard_normal((T, H, D))
+    A = rng.standard_normal((G, R, (H // G) * D))
+    Bm = rng.standard_normal((dm, G * R))
+    return o, A, Bm
+
+
+def test_grouped_out_proj_identity_is_concatenation():
+    """Identity group matrices (R = heads per group x D) and an identity dense matrix:
+    the projection returns the head outputs concatenated, exactly."""
+    T, H, D, G = 4, 8, 3, 2
+    o = np.random.default_rng(1).standard_normal((T, H, D))
+    Kg = (H // G) * D
+    A = np.stack([np.eye(Kg)] * G)
+    z, y = oracle.grouped_out_proj(o, A, np.eye(G * Kg), G)
+    assert np.array_equal(z, o.reshape(T, H * D)) and np.array_equal(y, o.reshape(T, H * D))
+
+
+def test_grouped_out_proj_one_group_is_two_matrix_products():
+    """G = 1 is the textbook chain of two dense projections, y = (o A^T) B^T (a library
+    matmul here); R differs from the group width, so a transposed operand cannot pass."""
+    o, A, Bm = _gop_case(2, G=1)
+    z, y = oracle.grouped_out_proj(o, A, Bm, 1)
+    z_ref = o.reshape(o.shape[0], -1) @ A[0].T
+    np.testing.assert_allclose(z, z_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(y, z_ref @ Bm.T, rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_out_proj_equals_block_diagonal_single_group():
+    """G groups equal one group whose matrix is block diagonal (group g's matrix on the
+    block of its heads): the grouping only removes the zero blocks."""
+    o, A, Bm = _gop_case(3)
+    G, R, Kg = A.shape
+    Abd = np.zeros((1, G * R, G * Kg))
+    for g in range(G):
+        Abd[0, g * R:(g + 1) * R, g * Kg:(g + 1) * Kg] = A[g]
+    z, y = oracle.grouped_out_proj(o, A, Bm, G)
+    z1, y1 = oracle.grouped_out_proj(o, Abd, Bm, 1)
+    np.testing.assert_allclose(z, z1, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(y, y1, rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_out_proj_group_locality_and_linearity():
+    """Changing the heads of group g changes only that group's R intermediate values; the
+    projection is linear in the head outputs."""
+    o, A, Bm = _gop_case(4)
+    G, R, _ = A.shape
+    H = o.shape[1]
+    z, y = oracle.grouped_out_proj(o, A, Bm, G)
+    for g in range(G):
+        o2 = o.copy()
+        o2[:, g * (H // G):(g + 1) * (H // G)] += 1.0
+        z2, _ = oracle.grouped_out_proj(o2, A, Bm, G)
+        changed = np.any(z2 != z, axis=0)
+        assert changed[g * R:(g + 1) * R].all() and not np.delete(changed, np.s_[g * R:(g + 1) * R]).any()
+    z3, y3 = oracle.grouped_out_proj(2.5 * o, A, Bm, G)
+    np.testing.assert_allclose(y3, 2.5 * y, rtol=1e-12, atol=1e-12)
