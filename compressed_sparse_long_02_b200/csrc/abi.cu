@@ -125,22 +125,8 @@ csa_status csa_compress(const csa_pool_cfg* cfg, int B, int T, const void* kv, c
   a.E_max = E_max;
   a.fp4 = fp4_out;
   a.fp4_scale = fp4_scale;
-  csa_status st = from_cuda(launch_pool(a, stream));
-  if (st != CSA_OK || window_kv == nullptr) return st;
-  NormRopeArgs w{};
-  w.x = kv;
-  w.in_bf16 = a.in_bf16;
-  w.rows = static_cast<int64_t>(B) * T;
-  w.heads = 1;
-  w.C = cfg->C;
-  w.pos = nullptr;
-  w.pos_mod = T;
-  w.norm = cfg->norm;
-  w.eps = cfg->eps;
-  w.rope_dims = cfg->rope_dims;
-  w.theta = cfg->rope_theta;
-  w.out = static_cast<uint16_t*>(window_kv);
-  return from_cuda(launch_norm_rope(w, stream));
+  a.window = static_cast<uint16_t*>(window_kv);  // written in the same pass as the entries
+  return from_cuda(launch_pool(a, stream));
 }
 
 csa_status csa_compress_step(const csa_pool_cfg* cfg, int B, const int32_t* pos, const void* kv, const void* logits,
@@ -433,6 +419,30 @@ csa_status hca_attn(int Nq, int H, int D, int mprime, int W, float scale, const 
   a.ws_bytes = ws_bytes;
   const int max_keys = E_max + (W < Tw ? W : Tw);
   return attn_common(a, max_keys, stream);
+}
+
+csa_status csa_grouped_out_proj(int T, int H, int D, int G, int R, int d_model, const void* o, const void* A,
+                                const void* Bm, void* z, void* y, cudaStream_t stream) {
+  if (T < 0 || H < 1 || D < 1 || G < 1 || R < 1 || d_model < 1 || H % G != 0) return CSA_ERR_INVALID_ARG;
+  if (((H / G) * static_cast<int64_t>(D)) % 64 != 0 || R % 256 != 0 || d_model % 256 != 0) return CSA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(H) * D * 2 > (int64_t(1) << 31) || static_cast<int64_t>(G) * R * 2 > (int64_t(1) << 31))
+    return CSA_ERR_UNSUPPORTED;
+  if (T == 0) return CSA_OK;
+  if (!o || !A || !Bm || !z || !y) return CSA_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(A) || !aligned16(Bm) || !aligned16(z) || !aligned16(y)) return CSA_ERR_ALIGNMENT;
+  GroupedProjArgs a{};
+  a.T = T;
+  a.H = H;
+  a.D = D;
+  a.G = G;
+  a.R = R;
+  a.d_model = d_model;
+  a.o = o;
+  a.A = A;
+  a.Bm = Bm;
+  a.z = static_cast<uint16_t*>(z);
+  a.y = static_cast<uint16_t*>(y);
+  return from_cuda(launch_grouped_out_proj(a, stream));
 }
 
 csa_status csa_get_device_error(int32_t* code_out, cudaStream_t stream) {

@@ -5,8 +5,8 @@
 //   E    = smallest integer with amax <= 6 * 2^E, clamped to [-127, 127]; amax == 0 -> -127
 //   code = round-half-even of x / 2^E onto {0, .5, 1, 1.5, 2, 3, 4, 6}; bit 3 = sign of x
 //   scale byte = E + 127; element 2i in the low nibble of byte i.
-// Every step is exact (power-of-two scaling, comparisons), so the bytes are a pure
-// function of the input bits.
+// Every step is exact (power-of-two scaling, comparisons or the hardware E2M1 rounding
+// of an exactly scaled value), so the bytes are a pure function of the input bits.
 #pragma once
 #include <cstdint>
 
@@ -41,6 +41,33 @@ __device__ __forceinline__ uint32_t e2m1_code(float x, float T) {
   return c | (signbit(x) ? 8u : 0u);
 }
 
+// 2^-E as a float, E in [-127, 127] (2^-127 is the subnormal 0x00400000)
+__device__ __forceinline__ float mx_pow2_neg(int E) { return mx_pow2(-E); }
+
+// The same codes through the hardware conversion: with y = x * 2^-E (exact: a power-of-two
+// scaling whose result is normal whenever it can round to a nonzero code, and a
+// subnormal y rounds to a signed zero either way), cvt.rn.satfinite.e2m1x2 rounds y to
+// the nearest E2M1 value, ties to the even code, which is the rule above; |y| <= 6 by the
+// choice of E, so saturation never acts.  Returns the byte (lo in bits 0-3, hi in 4-7).
+__device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 q;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q, %2, %1;\n\t"
+      "cvt.u32.u8 %0, q;\n\t}\n"
+      : "=r"(r)
+      : "f"(lo), "f"(hi));
+  return r;
+}
+
+// Eight values scaled by inv_T = 2^-E into four packed bytes (element 2i in the low nibble
+// of byte i).
+__device__ __forceinline__ uint32_t e2m1x8_rn(const float (&v)[8], float inv_T) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w |= e2m1x2_rn(v[2 * i] * inv_T, v[2 * i + 1] * inv_T) << (8 * i);
+  return w;
+}
+
 // Encode the pair (x0, x1) held by this thread, where 16 consecutive lanes (aligned
 // to 16) hold one 32-element block.  All 32 lanes of the warp must call it.
 __device__ __forceinline__ void mxfp4_encode_pair(float x0, float x1, uint8_t& byte, uint8_t& scale_byte) {
@@ -48,8 +75,8 @@ __device__ __forceinline__ void mxfp4_encode_pair(float x0, float x1, uint8_t& b
 #pragma unroll
   for (int o = 1; o < 16; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
   const int E = mx_block_exponent(am);
-  const float T = mx_pow2(E);
-  byte = static_cast<uint8_t>(e2m1_code(x0, T) | (e2m1_code(x1, T) << 4));
+  const float inv_T = mx_pow2_neg(E);
+  byte = static_cast<uint8_t>(e2m1x2_rn(x0 * inv_T, x1 * inv_T));
   scale_byte = static_cast<uint8_t>(E + 127);
 }
 
