@@ -18,7 +18,7 @@ import torch
 __all__ = ["CsaError", "lib", "csa_compress", "csa_compress_step", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk",
            "csa_index_score", "csa_index_score_q", "csa_topk_select",
            "csa_index_topk_workspace", "csa_sparse_attn", "csa_sparse_attn_workspace", "hca_attn",
-           "hca_attn_workspace", "csa_get_device_error", "csa_set_batch_invariant", "LIB_PATH", "DEVERR_NONE", "DEVERR_TIMEOUT",
+           "hca_attn_workspace", "csa_grouped_out_proj", "csa_get_device_error", "csa_set_batch_invariant", "LIB_PATH", "DEVERR_NONE", "DEVERR_TIMEOUT",
            "DEVERR_INDEX"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcsa.so")
@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
             L.hca_attn.argtypes = [I, I, I, I, I, F, P, P, P, I, I, P, P, I, P, P, P, P, P, SZ, P]
             L.hca_attn_workspace.argtypes = [I, I, I, I, I]
             L.hca_attn_workspace.restype = SZ
+            L.csa_grouped_out_proj.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P]
             L.csa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
             L.csa_set_batch_invariant.argtypes = [I]
             L.csa_set_batch_invariant.restype = I
@@ -75,7 +76,7 @@ def lib() -> ctypes.CDLL:
             for fn in ("csa_compress", "csa_compress_step", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk", "csa_index_score",
                        "csa_index_score_q",
                        "csa_topk_select", "csa_sparse_attn",
-                       "hca_attn", "csa_get_device_error"):
+                       "hca_attn", "csa_grouped_out_proj", "csa_get_device_error"):
                 getattr(L, fn).restype = I
             _lib = L
     return _lib
@@ -320,6 +321,23 @@ def hca_attn(q, q_pos, q_seq, entries, n_entries, window, window_base, *, mprime
                         _ptr(workspace), workspace.numel(), _stream(q))
     _check("hca_attn", st)
     return out, lse
+
+
+def csa_grouped_out_proj(o, A, Bm, *, z=None, y=None):
+    """Grouped output projection: o [T, H, D] bf16; A [G, R, (H/G) D] bf16; Bm [d_model, G R] bf16.
+    Returns (z [T, G R], y [T, d_model]) bf16."""
+    T, H, D = o.shape
+    G, R, Kg = A.shape
+    d_model = Bm.shape[0]
+    for t, nm in ((o, "o"), (A, "A"), (Bm, "Bm")):
+        _need(t, torch.bfloat16, None, nm)
+    if Kg * G != H * D or tuple(Bm.shape) != (d_model, G * R):
+        raise ValueError("inconsistent projection shapes")
+    z = torch.empty((T, G * R), dtype=torch.bfloat16, device=o.device) if z is None else z
+    y = torch.empty((T, d_model), dtype=torch.bfloat16, device=o.device) if y is None else y
+    st = lib().csa_grouped_out_proj(T, H, D, G, R, d_model, _ptr(o), _ptr(A), _ptr(Bm), _ptr(z), _ptr(y), _stream(o))
+    _check("csa_grouped_out_proj", st)
+    return z, y
 
 
 def csa_set_batch_invariant(on: bool) -> None:

@@ -99,6 +99,7 @@ struct PoolArgs {
   int E_max;
   uint8_t* fp4;       // nullable, [B, E_max, C/2]
   uint8_t* fp4_scale; // nullable, [B, E_max, C/32]
+  uint16_t* window;   // nullable, [B, T, C]: RoPE_u(RMSNorm(kv[u])) of every token (not in streaming mode)
   // Streaming (decode) mode when non-null: device [B], the position of each sequence's
   // newest token; kv / logits are then [B, (1+overlap)*m, C], row s holding token
   // pos - (1+overlap)*m + 1 + s, and only the entry that token completes is written.
@@ -166,5 +167,16 @@ size_t attn_workspace_bytes(int Nq, int H, int D, int max_keys);
 void set_batch_invariant(bool on);
 bool batch_invariant();
 cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s);
+
+// ---------------------------------------------------------------- grouped output projection
+struct GroupedProjArgs {
+  int T, H, D, G, R, d_model;
+  const void* o;   // bf16 [T, H * D]
+  const void* A;   // bf16 [G, R, (H / G) * D]
+  const void* Bm;  // bf16 [d_model, G * R]
+  uint16_t* z;     // bf16 [T, G * R]
+  uint16_t* y;     // bf16 [T, d_model]
+};
+cudaError_t launch_grouped_out_proj(const GroupedProjArgs& a, cudaStream_t s);
 
 }  // namespace csa

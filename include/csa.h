@@ -15,6 +15,7 @@
  *   csa_index_topk      lightning-indexer scores of every visible entry, then top-k.
  *   csa_sparse_attn     shared-KV MQA over the top-k entries plus the raw-token window.
  *   hca_attn            shared-KV MQA over every visible HCA entry plus the window.
+ *   csa_grouped_out_proj  grouped projection of the head outputs to the hidden size.
  *
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers unless marked "host".  The caller
@@ -281,6 +282,23 @@ CSA_API csa_status hca_attn(int Nq, int H, int D, int mprime, int W, float scale
                     const int32_t* n_entries, int Tw, const void* window_kv, const int32_t* window_base,
                     void* out, float* lse, void* workspace, size_t ws_bytes, cudaStream_t stream);
 CSA_API size_t hca_attn_workspace(int Nq, int H, int D, int E_max, int W);
+
+/*
+ * csa_grouped_out_proj -- grouped output projection of the core-attention outputs back to
+ * the hidden size ("DeepSeek-V4: Towards Highly Efficient Million-Token Context
+ * Intelligence", section 2.3, "Shared KV and output projection": CSA and HCA project their
+ * many head outputs through a grouped projection, cheaper than one dense projection).
+ * The H heads form G groups of H/G consecutive heads:
+ *   z[t, g R + r] = sum_i o[t, g (H/G) D + i] A[g, r, i]      (i < (H/G) D; group g's own matrix)
+ *   y[t, n]       = sum_j z[t, j] Bm[n, j]                    (j < G R)
+ * o bf16 [T, H, D] (the attention output layout); A bf16 [G, R, (H/G) D]; Bm bf16
+ * [d_model, G R]; z bf16 [T, G R] (the intermediate, written, caller-owned); y bf16
+ * [T, d_model].  float32 accumulation; z is rounded to bf16 before the second product.
+ * Supported: (H/G) D a multiple of 64, R and d_model multiples of 256.  Two tcgen05 GEMM
+ * launches on `stream`.
+ */
+CSA_API csa_status csa_grouped_out_proj(int T, int H, int D, int G, int R, int d_model, const void* o, const void* A,
+                                        const void* Bm, void* z, void* y, cudaStream_t stream);
 
 /* Synchronises `stream`, returns the device error word of the current device in
  * *code_out and clears it.  CSA_ERR_CUDA if the stream reports an error. */
