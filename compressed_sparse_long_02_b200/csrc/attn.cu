@@ -65,10 +65,21 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kSplitSMs = 148;             // B200 SM count used to size decode splits
 constexpr int kMaxSplits = 8;              // portable cluster size
 
+constexpr int kPBufs = 3;           // P buffers: 2 used by the interleaved pipeline, 3 by the two-pass one
+constexpr int kMaxTiles2 = kPBufs;  // tiles a CTA's share may have on the two-pass pipeline
+constexpr uint32_t kColO2 = 256;    // two-pass: S^T of up to 3 tiles in [0, 192), O^T in [256, 512)
+// Two-pass slab slots: the K pass cycles through the ring and the P buffers (the softmax
+// writes P only after the last QK), the V pass through the ring and Q's four 16 KB slabs
+// (free once the last QK has completed).  Barrier pairs: K slot s and V slot s < kRing
+// share pair s; V slot kRing + i uses pair kRing + kPBufs + i.
+constexpr int kSlotsK2 = kRing + kPBufs;
+constexpr int kSlotsV2 = kRing + 4;
+constexpr int kSlotBars = kRing + kPBufs + 4;
+static_assert(kSlotsV2 % 2 == 0, "V slabs go in adjacent pairs");
 constexpr size_t kOffQ = 0;                                       // 64 KB: [8 d-atoms][64 heads][128 B]
 constexpr size_t kOffRing = 64 * 1024;                            // kRing x 16 KB
-constexpr size_t kOffP = kOffRing + kRing * kSlabBytes;           // 2 x 16 KB: [128 keys][128 B] x 8 atoms
-constexpr size_t kOffSmall = kOffP + 2 * 16384;                   // reductions, stats, barriers
+constexpr size_t kOffP = kOffRing + kRing * kSlabBytes;           // kPBufs x 16 KB: [128 keys][128 B]
+constexpr size_t kOffSmall = kOffP + kPBufs * 16384;              // reductions, stats, barriers
 constexpr size_t kOffIdx = kOffSmall + 4096;                      // this CTA's slice of the index list
 constexpr int kIdxCap = 2048;
 constexpr size_t kAttnSmem = kOffIdx + 4 * kIdxCap + 1024;        // + alignment slack
@@ -92,6 +103,7 @@ struct AttnParams {
   float* part_o;   // [Nq, splits, H, D]
   float2* part_ml; // [Nq, splits, H]
   int rows_per_split, splits;
+  int two_pass;    // every CTA's share is at most kMaxTiles2 tiles: attend_2pass
   int32_t* err;
 };
 
@@ -101,20 +113,44 @@ struct KeyList {
   int64_t u_lo, wbase;
 };
 
-__device__ __forceinline__ KeyList key_list(const AttnParams& p, int n) {
+// The query's step metadata: its sequence (in range or not), position, window base and
+// (dense mode) entry count.  No kernel of this library writes these arrays, and a kernel
+// of the caller's that does never lets this one start before it completes (it does not
+// release its dependents early), so they are read before the wait on the previous grid.
+struct KeyMeta {
+  bool ok;
+  int b;
+  int64_t t, wbase, ne;
+};
+
+__device__ __forceinline__ KeyMeta key_meta(const AttnParams& p, int n) {
+  KeyMeta m{};
+  m.b = p.q_seq[n];
+  m.ok = m.b >= 0 && m.b < p.B;
+  if (m.ok) {
+    m.t = p.q_pos[n];
+    m.wbase = p.window_base[m.b];
+    m.ne = p.dense ? p.n_entries[m.b] : 0;
+  }
+  return m;
+}
+
+// The key list; in sparse mode the selection count comes from the previous grid (top-k),
+// so this runs after the wait.
+__device__ __forceinline__ KeyList key_list(const AttnParams& p, int n, const KeyMeta& m) {
   KeyList kl;
-  kl.b = p.q_seq[n];
-  const int64_t t = p.q_pos[n];
+  kl.b = m.b;
+  const int64_t t = m.t;
   if (p.dense) {
     int64_t v = (t + 1) / p.mprime;
     v = v < 0 ? 0 : v;
-    const int64_t ne = min(p.n_entries[kl.b], p.E_max);
+    const int64_t ne = min(m.ne, static_cast<int64_t>(p.E_max));
     kl.n_sel = static_cast<int>(v < ne ? v : ne);
   } else {
     const int c = p.cnt ? p.cnt[n] : 0;
     kl.n_sel = c < 0 ? 0 : (c > p.k ? p.k : c);
   }
-  kl.wbase = p.window_base[kl.b];
+  kl.wbase = m.wbase;
   int64_t lo = t - p.W + 1;
   if (lo < 0) lo = 0;
   if (lo < kl.wbase) lo = kl.wbase;
@@ -154,6 +190,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// 2^x by the hardware approximation (relative error ~2^-22; probabilities are rounded to
+// bf16 right after)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Stage st of the slab sequence K0 | K1 V0 | K2 V1 | ... | V(n-1): tile and pass.
 __device__ __forceinline__ void stage_of(int st, int n_tiles, int& tile, bool& is_v) {
   if (st == 0) {
@@ -183,15 +227,15 @@ struct AttnSmem {
   float* l_run;      // [64]
   float* alpha;      // [64]
   float* inv_l;      // [64]
-  uint8_t* row_ok;   // [2][128]: key row has a valid source
+  uint8_t* row_ok;   // [kPBufs][128]: key row has a valid source
   uint64_t* q_full;     // TMA: Q landed
-  uint64_t* full;       // [kRing] producers: slab landed
-  uint64_t* slot_free;  // [kRing] MMA commit: slab consumed
-  uint64_t* s_full;     // [2] MMA commit: S^T of a tile in TMEM
+  uint64_t* full;       // [kSlotBars] producers: slab landed
+  uint64_t* slot_free;  // [kSlotBars] MMA commit: slab consumed
+  uint64_t* s_full;     // [kPBufs] MMA commit: S^T of a tile in TMEM
   uint64_t* s_free;     // [2] softmax warps: S^T read
   uint64_t* p_full;     // [2] softmax warps: P written (and O^T rescaled)
   uint64_t* o_done;     // MMA commit: PV of a tile complete
-  uint64_t* row_ready;  // [2] producers: row_ok of a tile written
+  uint64_t* row_ready;  // [kPBufs] producers: row_ok of a tile written
   uint64_t* fin;        // MMA commit: every MMA of the CTA complete
   uint32_t* tmem_slot;
   volatile int* abort_flag;
@@ -207,16 +251,16 @@ struct AttnSmem {
     alpha = l_run + 64;
     inv_l = alpha + 64;
     row_ok = reinterpret_cast<uint8_t*>(inv_l + 64);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(row_ok + 256);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(row_ok + 128 * kPBufs);
     q_full = bars;
     full = q_full + 1;
-    slot_free = full + kRing;
-    s_full = slot_free + kRing;
-    s_free = s_full + 2;
+    slot_free = full + kSlotBars;
+    s_full = slot_free + kSlotBars;
+    s_free = s_full + kPBufs;
     p_full = s_free + 2;
     o_done = p_full + 2;
     row_ready = o_done + 1;
-    fin = row_ready + 2;
+    fin = row_ready + kPBufs;
     tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
     abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);
@@ -595,6 +639,343 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
   CSA_TB(3);
 }
 
+// Where slab j of the K pass and slab v of the V pass go: shared-memory offset, barrier
+// pair and the parity of the barrier phase (the use count of the pair, mod 2).
+struct Slot2 {
+  uint32_t off;
+  int bar;
+  uint32_t parity;
+};
+__device__ __forceinline__ Slot2 slot_k2(int j) {
+  const int sl = j % kSlotsK2;
+  Slot2 r;
+  r.off = sl < kRing ? static_cast<uint32_t>(kOffRing + sl * kSlabBytes) : static_cast<uint32_t>(kOffP + (sl - kRing) * kSlabBytes);
+  r.bar = sl;
+  r.parity = static_cast<uint32_t>(j / kSlotsK2) & 1u;
+  return r;
+}
+__device__ __forceinline__ Slot2 slot_v2(int v, int nK) {
+  const int sl = v % kSlotsV2;
+  Slot2 r;
+  if (sl < kRing) {
+    const int k_uses = nK > sl ? (nK - 1 - sl) / kSlotsK2 + 1 : 0;  // K slabs that used this pair
+    r.off = static_cast<uint32_t>(kOffRing + sl * kSlabBytes);
+    r.bar = sl;
+    r.parity = static_cast<uint32_t>(k_uses + v / kSlotsV2) & 1u;
+  } else {
+    r.off = static_cast<uint32_t>(kOffQ + (sl - kRing) * kSlabBytes);
+    r.bar = kRing + kPBufs + (sl - kRing);
+    r.parity = static_cast<uint32_t>(v / kSlotsV2) & 1u;
+  }
+  return r;
+}
+
+// Two-pass variant for a share of at most kMaxTiles2 tiles (decode: a query split over
+// several CTAs).  Slab order K0 | K1 | ... | K(n-1) | V0 | ... | V(n-1): the K pass is a
+// pure stream from HBM that QK consumes as slabs land (S^T of tile t in TMEM columns
+// 64 t), independent of the softmax; the softmax then runs once over every tile with
+// the exact maximum (no rescaling of O^T); the V pass re-gathers the same rows, now in
+// L2, into the ring slots the K pass frees, while the softmax works, and PV accumulates
+// O^T in columns [256, 512).  Same outputs as attend(): the normalised result or the
+// unnormalised partial with its (max, sum).
+__device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensorMap& tm_q, uint8_t* smem,
+                                             uint32_t tmem, int n, int split, const KeyList& kl, int row_begin,
+                                             int row_end, int n_tiles) {
+  const AttnSmem L(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tslot = blockIdx.x < 2 ? 4 + static_cast<int>(blockIdx.x) : -1;
+  if (threadIdx.x == 0) CSA_T(tslot, 0);
+  CSA_TB(2);
+
+  if (warp >= 8 && warp < 8 + kProdWarps) {
+    // ------------------------------------------------------------ gather producers
+    const int pw = warp - 8;
+    const int ptid = threadIdx.x - 256;
+    const int r0 = kRowsPerProd * pw;
+    const int nrows = min(kRowsPerProd, kBN - r0);
+    if (ptid == 0) {
+      mbar_arrive_expect_tx(L.q_full, kH * kD * 2);
+      for (int a = 0; a < 8; ++a) tma_load_2d(smem_u32(L.sQ + a * 8192), &tm_q, L.q_full, 128 * a, n * kH);
+    }
+    const int sel_here = max(0, min(row_end, kl.n_sel) - row_begin);
+    const bool staged = !p.dense && sel_here <= kIdxCap;
+    if (staged)
+      for (int i = lane; i < sel_here; i += 32)
+        if ((i % kBN) >= r0 && (i % kBN) < r0 + nrows) L.sidx[i] = p.idx[static_cast<size_t>(n) * p.k + row_begin + i];
+    __syncwarp();
+    auto row_src = [&](int tile, bool flag) -> const uint16_t* {
+      const int g = row_begin + tile * kBN + r0 + lane;
+      if (lane >= nrows || g >= row_end) return nullptr;
+      if (g < kl.n_sel) {
+        const int e = p.dense ? g : (staged ? L.sidx[g - row_begin] : p.idx[static_cast<size_t>(n) * p.k + g]);
+        if (e >= 0 && e < p.E_max) return p.entries + (static_cast<size_t>(kl.b) * p.E_max + e) * kD;
+        if (flag) atomicExch(p.err, CSA_DEVERR_INDEX);
+        return nullptr;
+      }
+      const int64_t u = kl.u_lo + (g - kl.n_sel);
+      return p.window + (static_cast<size_t>(kl.b) * p.Tw + static_cast<size_t>(u - kl.wbase)) * kD;
+    };
+    bool ok = true;
+    const int nK = kSlabs * n_tiles;
+    bool q_free = false;  // the last QK has completed: Q's slabs may take V slabs
+    for (int st = 0; ok && st < 2 * n_tiles; ++st) {
+      const bool is_v = st >= n_tiles;
+      const int tile = is_v ? st - n_tiles : st;
+      const uint16_t* src_row = row_src(tile, !is_v);
+      const bool valid = src_row != nullptr;
+      const unsigned long long src_ll = reinterpret_cast<unsigned long long>(valid ? src_row : p.entries);
+      if (ptid == 0) CSA_T(tslot, 8 + st);
+      if (!is_v && lane < nrows) {  // published before this tile's first slab is issued
+        L.row_ok[tile * 128 + r0 + lane] = valid ? 1 : 0;
+        mbar_arrive(&L.row_ready[tile]);
+      }
+      for (int ka = 0; ka < kSlabs; ++ka) {
+        const int j = is_v ? nK + tile * kSlabs + ka : tile * kSlabs + ka;  // slab sequence number
+        const Slot2 sl = is_v ? slot_v2(j - nK, nK) : slot_k2(j);
+        if (is_v && sl.bar >= kRing + kPBufs && !q_free) {
+          if (!warp_wait(&L.s_full[n_tiles - 1], 0, p.err, L.abort_flag)) {
+            ok = false;
+            break;
+          }
+          q_free = true;
+        }
+        if (!warp_wait(&L.slot_free[sl.bar], sl.parity ^ 1, p.err, L.abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (ptid == 0 && tslot == 4 && j < 64) CSA_T(10, j);
+        const uint32_t dst = smem_u32(smem + sl.off);
+        for (int qb = 0; qb < 8 * nrows; qb += 32) {
+          const int q = qb + lane;
+          const bool in = q < 8 * nrows;
+          const int rl = in ? q >> 3 : 0, c = q & 7;
+          const uint16_t* rs = reinterpret_cast<const uint16_t*>(__shfl_sync(0xffffffffu, src_ll, rl));
+          const bool rv = __shfl_sync(0xffffffffu, valid, rl);
+          if (in) cp_async_16(dst + sw128(r0 + rl, c), rs + (ka * 8 + c) * 8, rv);
+        }
+        cp_async_mbar_arrive_noinc(&L.full[sl.bar]);
+      }
+    }
+    cp_async_wait_all();
+    {
+      volatile int never = 0;
+      if (ptid == 0) mbar_wait(L.q_full, 0, p.err, &never);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_qk = idesc_bf16(128, kH, false, false);
+    constexpr uint32_t idesc_pv = idesc_bf16(128, kH, true, true);
+    const uint32_t base = smem_u32(smem), q0 = smem_u32(L.sQ), p0 = smem_u32(L.sP);
+    const int nK = kSlabs * n_tiles;
+    bool ok = warp_wait(L.q_full, 0, p.err, L.abort_flag);
+    if (lane == 0) CSA_T(tslot, 1);
+    for (int tile = 0; ok && tile < n_tiles; ++tile) {  // K pass: S^T[tile] = K Q^T
+      for (int ka = 0; ka < kSlabs; ++ka) {
+        const int j = tile * kSlabs + ka;
+        const Slot2 sl = slot_k2(j);
+        if (!warp_wait(&L.full[sl.bar], sl.parity, p.err, L.abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0 && tslot == 4 && j < 64) CSA_T(12, j);
+        fence_proxy_async_smem();
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + 64 * tile, smem_desc(base + sl.off + kk * 32, 16, 1024, kSwizzle128B),
+                     smem_desc(q0 + ka * 8192 + kk * 32, 16, 1024, kSwizzle128B), idesc_qk, (ka | kk) ? 1u : 0u);
+          tc_commit(&L.slot_free[sl.bar]);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        tc_commit(&L.s_full[tile]);
+        CSA_T(tslot, 24 + tile);
+      }
+      __syncwarp();
+    }
+    // V pass: O^T += V^T P^T[tile], a 128-dim chunk (two adjacent slots) at a time; tile t
+    // starts as soon as its P is written (the softmax publishes P tile by tile)
+    if (lane == 0) CSA_T(tslot, 30);
+    for (int tile = 0; ok && tile < n_tiles; ++tile) {
+      if (!warp_wait(&L.row_ready[tile], 1, p.err, L.abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      for (int dc = 0; dc < 4; ++dc) {
+        const int v = tile * kSlabs + 2 * dc;  // even: the chunk's two slabs sit in adjacent slots
+        const Slot2 s0 = slot_v2(v, nK), s1 = slot_v2(v + 1, nK);
+        if (!warp_wait(&L.full[s0.bar], s0.parity, p.err, L.abort_flag) ||
+            !warp_wait(&L.full[s1.bar], s1.parity, p.err, L.abort_flag)) {
+          ok = false;
+          break;
+        }
+        fence_proxy_async_smem();
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(tmem + kColO2 + 64 * dc, smem_desc(base + s0.off + ks * 2048, kSlabBytes, 1024, kSwizzle128B),
+                     smem_desc(p0 + tile * 16384 + ks * 2048, 16384, 1024, kSwizzle128B), idesc_pv,
+                     (tile > 0 || ks > 0) ? 1u : 0u);
+          tc_commit(&L.slot_free[s0.bar]);
+          tc_commit(&L.slot_free[s1.bar]);
+        }
+        __syncwarp();
+      }
+      if (lane == 0) CSA_T(tslot, 32 + tile);
+    }
+    if (ok && lane == 0) tc_commit(L.fin);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax (warps 0-7)
+    // thread = key row t of each tile (TMEM lane 32 (warp % 4) + lane) and 32 heads
+    const int q4 = warp & 3, hh = warp >> 2;
+    const int t = 32 * q4 + lane;
+    const int h0 = 32 * hh;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q4) << 16;
+    bool ok = true;
+    // sweep 1: the exact maximum of every head over the CTA's rows
+    float mx[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) mx[i] = -INFINITY;
+    for (int it = 0; it < n_tiles; ++it) {
+      const bool got = mbar_wait(&L.s_full[it], 0, p.err, L.abort_flag) &&
+                       mbar_wait(&L.row_ready[it], 0, p.err, L.abort_flag);
+      if (named_bar_or(1, 256, !got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (t == 0 && hh == 0) CSA_T(tslot, 40 + it);
+      const bool valid = row_begin + it * kBN + t < row_end && L.row_ok[it * 128 + t] != 0;
+      uint32_t sr[32];  // TMEM loads are warp-collective: every lane loads, invalid rows are masked
+      const uint32_t s_addr = tmem + lane_base + 64 * it + h0;
+      tmem_ld16(s_addr, sr);
+      tmem_ld16(s_addr + 16, sr + 16);
+      tmem_wait_ld();
+      if (valid) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx[i] = fmaxf(mx[i], __uint_as_float(sr[i]) * p.scale_log2);
+      }
+    }
+    if (ok) {
+      xreduce32<true>(mx);  // mx[0] = this warp's max of head h0 + lane
+      L.red_max[q4 * 64 + h0 + lane] = mx[0];
+      named_bar_sync(1, 256);
+      if (threadIdx.x < kH) {
+        const int h = threadIdx.x;
+        L.m_run[h] = fmaxf(fmaxf(L.red_max[h], L.red_max[64 + h]), fmaxf(L.red_max[128 + h], L.red_max[192 + h]));
+      }
+      named_bar_sync(1, 256);
+    }
+    // sweep 2: P = 2^(x - max) as bf16 per tile, and the per-thread sums
+    float lacc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) lacc[i] = 0.f;
+    for (int it = 0; ok && it < n_tiles; ++it) {
+      const bool valid = row_begin + it * kBN + t < row_end && L.row_ok[it * 128 + t] != 0;
+      float x[32];
+      uint32_t sr[32];
+      const uint32_t s_addr = tmem + lane_base + 64 * it + h0;
+      tmem_ld16(s_addr, sr);
+      tmem_ld16(s_addr + 16, sr + 16);
+      tmem_wait_ld();
+      if (valid) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const float4 mm = *reinterpret_cast<const float4*>(L.m_run + h0 + i);
+          x[i] = fast_exp2(fmaf(__uint_as_float(sr[i]), p.scale_log2, -mm.x));
+          x[i + 1] = fast_exp2(fmaf(__uint_as_float(sr[i + 1]), p.scale_log2, -mm.y));
+          x[i + 2] = fast_exp2(fmaf(__uint_as_float(sr[i + 2]), p.scale_log2, -mm.z));
+          x[i + 3] = fast_exp2(fmaf(__uint_as_float(sr[i + 3]), p.scale_log2, -mm.w));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) lacc[i] += x[i];
+      uint8_t* pb = L.sP + it * 16384;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint4 w4 = make_uint4(pack_bf16x2(x[8 * c], x[8 * c + 1]), pack_bf16x2(x[8 * c + 2], x[8 * c + 3]),
+                                    pack_bf16x2(x[8 * c + 4], x[8 * c + 5]), pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
+        *reinterpret_cast<uint4*>(pb + sw128(t, 4 * hh + c)) = w4;
+      }
+      // P of this tile is complete once all 256 threads' stores are: the tile's row_ready
+      // barrier, whose first phase the producers completed, takes its second phase from
+      // the 8 softmax warps (128 arrivals: 16 per warp)
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane < 16) mbar_arrive(&L.row_ready[it]);
+    }
+    if (t == 0 && hh == 0) CSA_T(tslot, 48);
+    // ------------------------------------------------------------ epilogue
+    CSA_TB(6);
+    const bool fin_ok = !named_bar_or(1, 256, !(ok && mbar_wait(L.fin, 0, p.err, L.abort_flag)));
+    ok = ok && fin_ok;
+    CSA_TB(7);
+    if (t == 0 && hh == 0) CSA_T(tslot, 2);
+    tc_fence_after();
+    xreduce32<false>(lacc);
+    L.red_sum[q4 * 64 + h0 + lane] = lacc[0];
+    named_bar_sync(1, 256);
+    if (threadIdx.x < kH) {
+      const int h = threadIdx.x;
+      L.l_run[h] = (L.red_sum[h] + L.red_sum[64 + h]) + (L.red_sum[128 + h] + L.red_sum[192 + h]);
+      L.inv_l[h] = L.l_run[h] > 0.f ? 1.0f / L.l_run[h] : 0.f;
+    }
+    named_bar_sync(1, 256);
+    if (ok) {
+#pragma unroll 1
+      for (int dp = 0; dp < 4; dp += 2) {
+        uint32_t o[2][32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t ta = tmem + lane_base + kColO2 + 64 * (dp + c) + h0;
+          tmem_ld16(ta, o[c]);
+          tmem_ld16(ta + 16, o[c] + 16);
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int d = (dp + c) * 128 + t;
+          if (p.splits == 1) {
+            uint16_t* ob = p.out + (static_cast<size_t>(n) * kH + h0) * kD + d;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const __nv_bfloat16 bv = __float2bfloat16_rn(__uint_as_float(o[c][i]) * L.inv_l[h0 + i]);
+              ob[i * kD] = *reinterpret_cast<const uint16_t*>(&bv);
+            }
+          } else {
+            float* pbo = p.part_o + ((static_cast<size_t>(n) * p.splits + split) * kH + h0) * kD + d;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pbo[i * kD] = __uint_as_float(o[c][i]);
+          }
+        }
+      }
+      if (threadIdx.x < kH) {
+        const int h = threadIdx.x;
+        const float l = L.l_run[h], m = L.m_run[h];
+        if (p.splits == 1) {
+          if (p.lse) p.lse[n * kH + h] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        } else {
+          p.part_ml[(static_cast<size_t>(n) * p.splits + split) * kH + h] = make_float2(l > 0.f ? m : -INFINITY, l);
+        }
+      }
+    } else if (threadIdx.x < kH && p.splits > 1) {
+      p.part_ml[(static_cast<size_t>(n) * p.splits + split) * kH + threadIdx.x] = make_float2(-INFINITY, 0.f);
+    }
+  }
+  if (threadIdx.x == 0) CSA_T(tslot, 3);
+  CSA_TB(3);
+}
+
 // Barriers, running statistics and the TMEM allocation: touches no global memory, so it
 // runs before the wait on the previous grid.  Returns the TMEM base address.
 __device__ __forceinline__ uint32_t attn_setup(uint8_t* smem) {
@@ -615,15 +996,17 @@ __device__ __forceinline__ uint32_t attn_setup(uint8_t* smem) {
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < kRing; ++i) {
+    for (int i = 0; i < kSlotBars; ++i) {
       mbar_init(&full[i], kProdThreads);
       mbar_init(&slot_free[i], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kPBufs; ++b) {
       mbar_init(&s_full[b], 1);
+      mbar_init(&row_ready[b], kBN);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&s_free[b], 8);
       mbar_init(&p_full[b], 8);
-      mbar_init(&row_ready[b], kBN);
     }
     mbar_init(o_done, 1);
     mbar_init(fin, 1);
@@ -714,23 +1097,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   if (threadIdx.x == 0) prefetch_tmap(&tm_q);
   const uint32_t tmem = attn_setup(smem);
-  griddep_enter();
-  CSA_TB(1);
   const int n = blockIdx.x / p.splits;
   const int split = blockIdx.x % p.splits;  // the CTA's rank in its cluster when splits > 1
-  const bool seq_ok = p.q_seq[n] >= 0 && p.q_seq[n] < p.B;  // same for every CTA of the query (cluster)
+  const KeyMeta meta = key_meta(p, n);
+  griddep_enter();
+  CSA_TB(1);
+  const bool seq_ok = meta.ok;  // same for every CTA of the query (cluster)
   if (!seq_ok && threadIdx.x == 0 && split == 0) atomicExch(p.err, CSA_DEVERR_INDEX);
   KeyList kl{};
   int row_begin = 0, row_end = 0, n_tiles = 0;
   if (seq_ok) {
-    kl = key_list(p, n);
+    kl = key_list(p, n, meta);
     const int nk = kl.n_sel + kl.n_win;
     row_begin = split * p.rows_per_split;
     row_end = min(nk, row_begin + p.rows_per_split);
     n_tiles = row_end > row_begin ? (row_end - row_begin + kBN - 1) / kBN : 0;
   }
 
-  if (n_tiles > 0) attend(p, tm_q, smem, tmem, n, split, kl, row_begin, row_end, n_tiles);
+  if (n_tiles > 0) {
+    if (p.two_pass)
+      attend_2pass(p, tm_q, smem, tmem, n, split, kl, row_begin, row_end, n_tiles);
+    else
+      attend(p, tm_q, smem, tmem, n, split, kl, row_begin, row_end, n_tiles);
+  }
   tc_fence_before();
   __syncthreads();
   if ((threadIdx.x >> 5) == kMmaWarp) {
@@ -834,6 +1223,7 @@ cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s) {
   const int splits = split_count(a.Nq, max_keys);
   p.splits = splits;
   p.rows_per_split = std::max(32, (((max_keys + splits - 1) / splits) + 31) / 32 * 32);
+  p.two_pass = p.rows_per_split <= kMaxTiles2 * kBN ? 1 : 0;
   if (static_cast<int64_t>(a.Nq) * kH >= INT32_MAX) return cudaErrorInvalidValue;  // 32-bit TMA row coordinate
   CUtensorMap tm_q;  // the queries as 64-row x 128-byte boxes
   if (!encode_2d_u8(&tm_q, a.q, kD * 2, static_cast<uint64_t>(a.Nq) * kH, 128, kH, CU_TENSOR_MAP_SWIZZLE_128B))
