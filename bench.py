@@ -48,6 +48,44 @@ def load_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# ----------------------------------------------------------------------------- tensor peaks
+FP4_DATASHEET_TFLOPS = 9000.0  # NVIDIA B200 dense FP4 (the 18 PFLOP/s figure is with 2:4 sparsity)
+
+
+def measure_tensor_peaks(dev, reps: int = 3) -> dict:
+    """Dense tcgen05 rates of this GPU from the library's throughput probe (one CTA per SM,
+    M = 128, N = 256, operands resident in shared memory): kind::mxf4 block-scaled FP4,
+    the denominator of the FP4 indexer, and kind::f16 bf16 for comparison with the
+    library GEMM's measured bf16 rate.  Best of `reps` launches of a few ms each."""
+    import ctypes
+    import torch
+    from compressed_sparse_long_02_b200 import binding as B
+    L = B.lib()
+    L.csa_mma_peak_probe.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                     ctypes.POINTER(ctypes.c_double), ctypes.c_void_p]
+    L.csa_mma_peak_probe.restype = ctypes.c_int
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    out = {}
+    for name, mxf4, iters in (("mxf4", 1, 20000), ("bf16", 0, 40000)):
+        best = 0.0
+        for r in range(reps + 1):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flops = ctypes.c_double(0.0)
+            s.record()
+            st = L.csa_mma_peak_probe(mxf4, 256, iters, sms, ctypes.byref(flops), stream)
+            e.record()
+            torch.cuda.synchronize()
+            assert st == 0, f"csa_mma_peak_probe: status {st}"
+            if r > 0:  # the first launch warms up
+                best = max(best, flops.value / (s.elapsed_time(e) / 1e3) / 1e12)
+        out[name] = round(best, 1)
+    assert B.csa_get_device_error() == 0
+    return {"mxf4_tflops": out["mxf4"], "bf16_tflops_probe": out["bf16"], "ctas": sms,
+            "how": "tcgen05 M=128 N=256, operands in shared memory, one CTA per SM, best of 3",
+            "mxf4_datasheet_tflops": FP4_DATASHEET_TFLOPS}
+
+
 # ----------------------------------------------------------------------------- ncu traffic
 # DRAM bytes (read + write) per launch from one `ncu --set full` capture of the 128K
 # decode step (profiles/*_decode_128k.md), keyed by the sha1 of the kernel's source file
@@ -247,18 +285,19 @@ def capture_step(fn):
     return g
 
 
-def bench_decode(args, dist, peaks):
+def bench_decode(args, dist, peaks, name: str = "csa_decode_128k", e2e: bool = True, steps: int | None = None):
     import torch
     from compressed_sparse_long_02_b200 import binding as B
     from compressed_sparse_long_02_b200 import synth
-    wl = synth.WORKLOADS["csa_decode_128k"]
+    wl = synth.WORKLOADS[name]
+    steps = args.steps if steps is None else steps
     dev = torch.device("cuda", dist.local_rank)
     R = args.replicas
-    caches, steps, ws = setup_decode(wl, dev, R)
+    caches, step_inputs, ws = setup_decode(wl, dev, R)
     for i in range(R):  # eager pass: sets kernel attributes before capture
-        decode_step(wl, caches[i], steps[i], ws)
+        decode_step(wl, caches[i], step_inputs[i], ws)
     torch.cuda.synchronize()
-    graphs = [capture_step(lambda i=i: decode_step(wl, caches[i], steps[i], ws)) for i in range(R)]
+    graphs = [capture_step(lambda i=i: decode_step(wl, caches[i], step_inputs[i], ws)) for i in range(R)]
     for i in range(args.warmup):
         graphs[i % R].replay()
     torch.cuda.synchronize()
@@ -270,7 +309,7 @@ def bench_decode(args, dist, peaks):
     dist.barrier()
     torch.cuda.synchronize()
     start.record()
-    for i in range(args.steps):
+    for i in range(steps):
         graphs[i % R].replay()
     end.record()
     torch.cuda.synchronize()
@@ -282,22 +321,22 @@ def bench_decode(args, dist, peaks):
 
     # per-call device time: the same steps run eagerly behind a GPU sleep, so that the
     # calls queue up and execute back to back between the events
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    for i in range(args.steps):
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for i in range(steps):
         torch.cuda._sleep(2_000_000)
-        decode_step(wl, caches[i % R], steps[i % R], ws, evs[i])
+        decode_step(wl, caches[i % R], step_inputs[i % R], ws, evs[i])
     torch.cuda.synchronize()
     per = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in
            enumerate(["quantize", "index_score", "topk_select", "attention"])}
     nb = decode_bytes_per_query(wl)
     queries_per_step = wl.B * dist.world
-    value = queries_per_step * args.steps / (ms / 1e3)
-    ms_step = ms / args.steps
+    value = queries_per_step * steps / (ms / 1e3)
+    ms_step = ms / steps
     dom = max(per, key=per.get)
     dom_bytes = {"index_score": nb["index_score"], "attention": nb["attention"],
                  "quantize": wl.Hi * wl.Di * 4, "topk_select": wl.E * 4}[dom] * wl.B
     achieved = dom_bytes / (per[dom] / 1e3) / 1e9
-    step_gbs = nb["step"] * wl.B / (ms_local / args.steps / 1e3) / 1e9
+    step_gbs = nb["step"] * wl.B / (ms_local / steps / 1e3) / 1e9
     res = {
         "value": value, "ms_per_step": ms_step,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
@@ -307,11 +346,12 @@ def bench_decode(args, dist, peaks):
                           "frac": round(step_gbs / peaks["hbm_gbs"], 4)},
         "per_call_us": {k: round(v * 1e3, 2) for k, v in per.items()},
         "clocks": clk,
-        "gpu_launches": args.steps * 4,  # query encoding, indexer, top-k, attention (split merge inside)
+        "gpu_launches": steps * 4,  # query encoding, indexer, top-k, attention (split merge inside)
         "graph": "one CUDA graph per input replica, replayed back to back",
     }
-    res["e2e"] = bench_decode_e2e(args, wl, caches, steps, ws, dist)
-    del graphs, caches, steps, ws
+    if e2e:
+        res["e2e"] = bench_decode_e2e(args, wl, caches, step_inputs, ws, dist)
+    del graphs, caches, step_inputs, ws
     torch.cuda.empty_cache()
     return wl, res
 
@@ -412,7 +452,74 @@ def _dev_inputs(inp, dev):
     return out
 
 
-def bench_prefill(name, steps, warmup, dist, peaks):
+def prefill_calls(wl, t, dev):
+    """The prefill layer's C-ABI calls in the order the layer issues them, as (name, fn)
+    pairs (the indexer's scoring and top-k as the two calls csa_index_topk is made of, so
+    each is timed on its own)."""
+    import torch
+    from compressed_sparse_long_02_b200 import binding as B
+    T, E = wl.T, wl.E
+    pos = torch.arange(T, dtype=torch.int32, device=dev)
+    seq = torch.zeros(T, dtype=torch.int32, device=dev)
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    ne = torch.tensor([E], dtype=torch.int32, device=dev)
+    st = {}
+    kw = dict(m=wl.m, overlap=wl.overlap, norm=wl.norm, eps=wl.eps, rope_dims=wl.rope_dims, theta=wl.theta)
+    calls = [("compress_kv", lambda: st.__setitem__("pool", B.csa_compress(t["kv"], t["z"], t["bias"], want_window=True,
+                                                                            **kw)))]
+    if wl.kind == "csa_prefill":
+        E_pad = max(8, (E + 7) // 8 * 8)
+        calls += [
+            ("compress_ki", lambda: st.__setitem__("keys", B.csa_compress(
+                t["ki"], t["zi"], t["bias_i"], m=wl.m, overlap=wl.overlap, norm=False, want_entries=False,
+                want_fp4=True, E_max=E_pad))),
+            ("quantize_qi", lambda: st.__setitem__("qq", B.csa_quantize_mxfp4(t["qi"][0]))),
+        ]
+    calls.append(("norm_rope_q", lambda: st.__setitem__("q", B.csa_norm_rope(
+        t["q"][0], pos, norm=wl.norm, eps=wl.eps, rope_dims=wl.rope_dims, theta=wl.theta))))
+    if wl.kind == "csa_prefill":
+        w = t["w"][0].contiguous()
+        scores = torch.empty((T, max(8, (E + 7) // 8 * 8)), dtype=torch.float32, device=dev)  # no fill inside the timing
+        calls += [
+            ("index_score", lambda: st.__setitem__("scores", B.csa_index_score(
+                st["qq"][0], st["qq"][1], w, pos, seq, st["keys"]["fp4"], st["keys"]["fp4_scale"], ne, m=wl.m,
+                scores=scores))),
+            ("topk_select", lambda: st.__setitem__("sel", B.csa_topk_select(
+                st["scores"], pos, seq, ne, k=wl.k, m=wl.m, E_max=st["keys"]["fp4"].shape[1]))),
+            ("attention", lambda: st.__setitem__("out", B.csa_sparse_attn(
+                st["q"], pos, seq, st["pool"]["entries"], st["sel"][0], st["sel"][1], st["pool"]["window"], zero,
+                W=wl.W)[0])),
+        ]
+    else:
+        calls.append(("attention", lambda: st.__setitem__("out", B.hca_attn(
+            st["q"], pos, seq, st["pool"]["entries"], ne, st["pool"]["window"], zero, mprime=wl.m, W=wl.W)[0])))
+    return calls
+
+
+def prefill_work(wl) -> dict:
+    """Algorithmic work of each prefill call: (bound, amount, unit) with bytes for the
+    HBM-bound calls (compulsory traffic: inputs read once, outputs written once) and
+    dense FLOPs for the contractions."""
+    T, C, E, H, s = wl.T, wl.C, wl.E, wl.H, (2 if wl.dtype == "bf16" else 4)
+    w = {"compress_kv": ("hbm", 2 * T * C * s + E * C * 2 + T * C * 2),  # kv, z in; entries, window rows out
+         "norm_rope_q": ("hbm", T * H * C * (s + 2))}
+    if wl.kind == "csa_prefill":
+        Hi, Di = wl.Hi, wl.Di
+        vis = sum(min((t + 1) // wl.m, E) for t in range(T))
+        w["compress_ki"] = ("hbm", 2 * T * Di * s + E * (Di // 2 + Di // 32))
+        w["quantize_qi"] = ("hbm", T * Hi * Di * s + T * Hi * (Di // 2 + Di // 32))
+        w["index_score"] = ("tensor_fp4", indexer_flops(wl))
+        w["topk_select"] = ("hbm", vis * 4 + T * wl.k * 4 + T * 4)
+    w["attention"] = ("tensor_bf16", attention_flops(wl))
+    return w
+
+
+def bench_prefill(name, steps, warmup, dist, peaks, tensor_peaks):
+    """One prefill workload: the whole layer per step (tok/s), then every call timed on
+    its own (the calls queued behind a GPU sleep so that they run back to back between
+    events), each against its roofline: HBM for the memory-bound calls, the measured
+    bf16 library-GEMM burst peak for attention, the measured tcgen05 mxf4 rate for the
+    FP4 indexer (burst figures: each call is timed alone)."""
     import torch
     from compressed_sparse_long_02_b200 import binding as B
     from compressed_sparse_long_02_b200 import layer, synth
@@ -432,57 +539,94 @@ def bench_prefill(name, steps, warmup, dist, peaks):
     torch.cuda.synchronize()
     ms = dist.max(s.elapsed_time(e)) / steps
     assert B.csa_get_device_error() == 0
-    # dominant kernel: the attention call, timed alone on the same inputs
-    r = run(wl, t)
+    calls = prefill_calls(wl, t, dev)
+    for _, fn in calls:  # warm the call sequence once
+        fn()
     torch.cuda.synchronize()
-    seq = torch.zeros(wl.T, dtype=torch.int32, device=dev)
-    pos = torch.arange(wl.T, dtype=torch.int32, device=dev)
-    zero = torch.zeros(1, dtype=torch.int32, device=dev)
-    ne = torch.tensor([wl.E], dtype=torch.int32, device=dev)
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = max(1, steps)
-    a0.record()
-    for _ in range(reps):
-        if wl.kind == "csa_prefill":
-            B.csa_sparse_attn(r["q"], pos, seq, r["entries"], r["idx"], r["cnt"], r["window"], zero, W=wl.W,
-                              out=r["out"])
+    reps = max(2, steps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(reps)]
+    for r in range(reps):
+        torch.cuda._sleep(20_000_000)
+        evs[r][0].record()
+        for j, (_, fn) in enumerate(calls):
+            fn()
+            evs[r][j + 1].record()
+    torch.cuda.synchronize()
+    assert B.csa_get_device_error() == 0
+    per_us = {n: statistics.median(1e3 * ev[j].elapsed_time(ev[j + 1]) for ev in evs) for j, (n, _) in
+              enumerate(calls)}
+    work = prefill_work(wl)
+    per_call = {}
+    for n, us in per_us.items():
+        bound, amount = work[n]
+        if bound == "hbm":
+            ach = amount / (us / 1e6) / 1e9
+            per_call[n] = {"us": round(us, 2), "bound": "hbm", "algorithmic_bytes": amount, "achieved": round(ach, 1),
+                           "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4)}
         else:
-            B.hca_attn(r["q"], pos, seq, r["entries"], ne, r["window"], zero, mprime=wl.m, W=wl.W, out=r["out"])
-    a1.record()
-    torch.cuda.synchronize()
-    attn_ms = a0.elapsed_time(a1) / reps
-    flops = attention_flops(wl)
-    tf = flops / (attn_ms / 1e3) / 1e12
+            pk = tensor_peaks["mxf4_tflops"] if bound == "tensor_fp4" else peaks["bf16_tflops"]
+            ach = amount / (us / 1e6) / 1e12
+            per_call[n] = {"us": round(us, 2), "bound": "tensor", "algorithmic_flops": amount,
+                           "achieved": round(ach, 1), "unit": "TFLOP/s", "frac": round(ach / pk, 4),
+                           "peak": pk}
+    att = per_call["attention"]
     out = {"workload": name, "tokens": wl.T, "tok_per_s": wl.T * dist.world / (ms / 1e3), "ms_per_step": ms,
-           "roofline": {"bound": "tensor", "kernel": "attention", "achieved": round(tf, 1),
-                        "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                        "frac": round(tf / peaks["bf16_tflops_sustained"], 4), "attention_ms": round(attn_ms, 4),
-                        "algorithmic_flops": flops}}
+           "roofline": {"bound": "tensor", "kernel": "attention", "achieved": att["achieved"],
+                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": att["frac"],
+                        "attention_ms": round(att["us"] / 1e3, 4), "algorithmic_flops": att["algorithmic_flops"],
+                        "peak_source": "measured bf16 library GEMM, burst (the call is timed alone)"},
+           "per_call": per_call,
+           "per_call_sum_us": round(sum(per_us.values()), 1)}
     if wl.kind == "csa_prefill":
-        # the indexer's scoring alone: MXFP4 contraction of every visible (query, entry) pair
-        scores = torch.empty((wl.T, r["k_fp4"].shape[1]), dtype=torch.float32, device=dev)
-        for _ in range(2):
-            B.csa_index_score(r["q_fp4"], r["q_scale"], r["w"], pos, seq, r["k_fp4"], r["k_scale"], r["n_ent"], m=wl.m,
-                              scores=scores)
-        i0, i1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        i0.record()
-        for _ in range(reps):
-            B.csa_index_score(r["q_fp4"], r["q_scale"], r["w"], pos, seq, r["k_fp4"], r["k_scale"], r["n_ent"], m=wl.m,
-                              scores=scores)
-        i1.record()
-        torch.cuda.synchronize()
-        idx_ms = i0.elapsed_time(i1) / reps
-        iflops = indexer_flops(wl)
-        itf = iflops / (idx_ms / 1e3) / 1e12
-        fp4_peak = peaks["bf16_tflops"] * 4.0  # nominal dense fp4 / bf16 ratio (9 / 2.25) on the measured burst
-        out["indexer"] = {"bound": "tensor", "kernel": "index_score", "achieved": round(itf, 1),
-                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(itf / fp4_peak, 4),
-                          "index_ms": round(idx_ms, 4), "algorithmic_flops": iflops,
-                          "peak_source": "measured bf16 burst x 4 (nominal MXFP4 / bf16 ratio)"}
-        del scores
-    del t, r
+        ix = per_call["index_score"]
+        out["indexer"] = {"bound": "tensor", "kernel": "index_score", "achieved": ix["achieved"],
+                          "peak": tensor_peaks["mxf4_tflops"], "unit": "TFLOP/s", "frac": ix["frac"],
+                          "frac_of_datasheet": round(ix["achieved"] / tensor_peaks["mxf4_datasheet_tflops"], 4),
+                          "index_ms": round(ix["us"] / 1e3, 4), "algorithmic_flops": ix["algorithmic_flops"],
+                          "peak_source": "measured: tcgen05 kind::mxf4 probe (csa_mma_peak_probe)"}
+    del t, calls
     torch.cuda.empty_cache()
     return out
+
+
+def bench_out_proj(dist, peaks, reps: int = 5) -> dict:
+    """The grouped output projection at the 8K prefill's size (8192 tokens, 64 heads of
+    512 in 8 groups, R = 1024, hidden 4096): both tcgen05 GEMM stages of one call, timed
+    alone with events, against the measured bf16 library-GEMM burst peak."""
+    import torch
+    from compressed_sparse_long_02_b200 import binding as B
+    from compressed_sparse_long_02_b200 import synth
+    ps = synth.PROJ["csa_prefill_8k"]
+    dev = torch.device("cuda", dist.local_rank)
+    d = synth.proj_inputs_torch(ps, dev)
+    z = torch.empty((ps.T, ps.G * ps.R), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((ps.T, ps.d_model), dtype=torch.bfloat16, device=dev)
+    for _ in range(2):
+        B.csa_grouped_out_proj(d["o"], d["A"], d["Bm"], z=z, y=y)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        B.csa_grouped_out_proj(d["o"], d["A"], d["Bm"], z=z, y=y)
+    e.record()
+    torch.cuda.synchronize()
+    assert B.csa_get_device_error() == 0
+    ms = s.elapsed_time(e) / reps
+    flops = out_proj_flops(ps)
+    tf = flops / (ms / 1e3) / 1e12
+    del d, z, y
+    torch.cuda.empty_cache()
+    return {"workload": "grouped_out_proj_8k", "tokens": ps.T, "heads": ps.H, "head_dim": ps.D, "groups": ps.G,
+            "group_rank": ps.R, "d_model": ps.d_model, "ms": round(ms, 4), "tok_per_s": ps.T / (ms / 1e3),
+            "roofline": {"bound": "tensor", "kernel": "gemm_bf16 (two stages)", "achieved": round(tf, 1),
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
+                         "algorithmic_flops": flops,
+                         "peak_source": "measured bf16 library GEMM, burst (the call is timed alone)"}}
+
+
+def out_proj_flops(ps) -> float:
+    """2 x T x (H D R   (each group: (H/G) D inputs x R outputs, G groups)  +  G R d_model)."""
+    return 2.0 * ps.T * (ps.H * ps.D * ps.R + ps.G * ps.R * ps.d_model)
 
 
 def indexer_flops(wl) -> float:
@@ -526,6 +670,30 @@ def cpu_oracle_decode(wl, n_seq: int, budget_s: float = 12.0, seed_replica: int 
     return {"value": done / t_used, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{done} decode queries over {n_seq} sequences (full {wl.E}-entry caches, k={wl.k}, "
                       f"W={wl.W}), {chunk} in parallel, {t_used:.1f} s"}
+
+
+def cpu_oracle_single_thread(wl, n_query: int = 4, timeout_s: float = 240.0) -> dict:
+    """The same oracle decode on one thread: a child process with OMP_NUM_THREADS=1 (the
+    oracle's OpenMP pool is sized when the library loads, so this process cannot shrink
+    its own) runs `n_query` decode queries of full caches and reports queries/s."""
+    code = ("import json, sys, time; sys.path.insert(0, %r)\n"
+            "import oracle\nfrom compressed_sparse_long_02_b200 import synth\n"
+            "wl = synth.WORKLOADS['csa_decode_128k']\n"
+            "d = synth.decode_inputs(wl, B=%d)\n"
+            "kp, ks = oracle.mxfp4_quantize(d['ki'])\n"
+            "t0 = time.perf_counter()\n"
+            "qp, qs = oracle.mxfp4_quantize(d['qi'])\n"
+            "oracle.csa_decode(wl, d['entries'], kp, ks, d['q'], qp, qs, d['w'], d['window'], d['pos'])\n"
+            "print(json.dumps({'s': time.perf_counter() - t0}))\n") % (ROOT, n_query)
+    env = dict(os.environ, OMP_NUM_THREADS="1", CUDA_VISIBLE_DEVICES="")
+    try:
+        r = subprocess.run([sys.executable, "-c", code], env=env, cwd=ROOT, capture_output=True, text=True,
+                           timeout=timeout_s)
+        t = json.loads(r.stdout.strip().splitlines()[-1])["s"]
+    except Exception as e:  # a baseline figure, never a reason to fail the benchmark
+        return {"value": None, "unit": UNIT, "cores": 1, "error": str(e)[:200]}
+    return {"value": n_query / t, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n_query} decode queries (full {wl.E}-entry caches), OMP_NUM_THREADS=1, {t:.1f} s"}
 
 
 def run_reference(args, dist):
@@ -599,11 +767,22 @@ def main():
                 "step_roofline": res["step_roofline"], "per_call_us": res["per_call_us"], "e2e": res["e2e"],
                 "clocks": res["clocks"], "gpu_launches": res["gpu_launches"], "launch": res["graph"]}
         if not args.no_secondary:
-            sec_steps = 5
-            line["prefill"] = bench_prefill("csa_prefill_8k", sec_steps, 2, dist, peaks)
-            line["hca_prefill"] = bench_prefill("hca_prefill_64k", 3, 1, dist, peaks)
+            dev = torch.device("cuda", dist.local_rank)
+            tp = measure_tensor_peaks(dev)
+            line["tensor_peaks"] = tp
+            wl1, r1 = bench_decode(args, dist, peaks, name="csa_decode_1m", e2e=False, steps=min(args.steps, 20))
+            line["decode_1m"] = {"workload": "csa_decode_1m", "sequences_per_gpu": wl1.B, "context": wl1.L,
+                                 "entries": wl1.E, "value": r1["value"], "unit": UNIT, "ms_per_step": r1["ms_per_step"],
+                                 "step_roofline": r1["step_roofline"], "roofline": r1["roofline"],
+                                 "per_call_us": r1["per_call_us"], "clocks": r1["clocks"]}
+            line["gpu_launches_decode_1m"] = r1["gpu_launches"]
+            line["prefill"] = bench_prefill("csa_prefill_8k", 5, 2, dist, peaks, tp)
+            line["hca_prefill"] = bench_prefill("hca_prefill_64k", 3, 1, dist, peaks, tp)
+            line["out_proj"] = bench_out_proj(dist, peaks)
         if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
-            line["cpu_baseline"] = cpu_oracle_decode(wl, n_seq=min(wl.B, max(4, os.cpu_count() or 4)))
+            cb = cpu_oracle_decode(wl, n_seq=min(wl.B, max(4, os.cpu_count() or 4)))
+            cb["single_thread"] = cpu_oracle_single_thread(wl)
+            line["cpu_baseline"] = cb
         if dist.rank == 0:
             print(json.dumps(line), flush=True)
     finally:
