@@ -212,6 +212,7 @@ def decode_bytes_per_query(wl) -> dict:
     score_out = E * 4
     return {"step": keys + qi + gathered + window + q_o + idx,
             "index_score": keys + Hi * (Di // 2 + Di // 32) + Hi * 4 + score_out,
+            "index_topk": keys + Hi * (Di // 2 + Di // 32) + Hi * 4 + idx + 4,
             "attention": gathered + window + q_o + idx,
             "keys": keys}
 
@@ -233,7 +234,7 @@ def setup_decode(wl, dev, replicas: int):
     torch.cuda.synchronize()
     Bn = wl.B
     ws = {
-        "scores": torch.empty((Bn, wl.E), dtype=torch.float32, device=dev),
+        "index_ws": torch.empty(B.csa_index_topk_workspace(Bn, wl.E, wl.k), dtype=torch.uint8, device=dev),
         "idx": torch.empty((Bn, wl.k), dtype=torch.int32, device=dev),
         "cnt": torch.empty((Bn,), dtype=torch.int32, device=dev),
         "seq": torch.arange(Bn, dtype=torch.int32, device=dev),
@@ -246,10 +247,15 @@ def setup_decode(wl, dev, replicas: int):
     return caches, steps, ws
 
 
+DECODE_CALLS = ["quantize", "index_topk", "attention"]
+
+
 def decode_step(wl, cache, step, ws, ev=None):
-    """One decode step as four C-ABI calls; `ev` (optional) gets CUDA events between calls.
-    (csa_index_score_q would encode the queries inside the indexer instead, but with nine
-    indexer CTAs per query that repeats the encoding nine times; one encoding pass is
+    """One decode step as three C-ABI calls (query encoding, indexer + top-k, attention);
+    `ev` (optional) gets CUDA events between calls.  csa_index_topk runs one fused kernel
+    at the 128K shape (scores kept on chip) and the scoring and top-k kernels otherwise.
+    (csa_index_score_q would encode the queries inside the indexer instead, but with
+    several indexer CTAs per query that repeats the encoding; one encoding pass is
     cheaper here.)"""
     from compressed_sparse_long_02_b200 import binding as B
     if ev is not None:
@@ -257,18 +263,14 @@ def decode_step(wl, cache, step, ws, ev=None):
     B.csa_quantize_mxfp4(step["qi"], ws["q_fp4"], ws["q_scale"])
     if ev is not None:
         ev[1].record()
-    B.csa_index_score(ws["q_fp4"], ws["q_scale"], step["w"], step["pos"], ws["seq"], cache["k_fp4"],
-                      cache["k_scale"], cache["n_entries"], m=wl.m, scores=ws["scores"])
+    B.csa_index_topk(ws["q_fp4"], ws["q_scale"], step["w"], step["pos"], ws["seq"], cache["k_fp4"], cache["k_scale"],
+                     cache["n_entries"], k=wl.k, m=wl.m, workspace=ws["index_ws"], idx=ws["idx"], cnt=ws["cnt"])
     if ev is not None:
         ev[2].record()
-    B.csa_topk_select(ws["scores"], step["pos"], ws["seq"], cache["n_entries"], k=wl.k, m=wl.m, E_max=wl.E,
-                      idx=ws["idx"], cnt=ws["cnt"])
-    if ev is not None:
-        ev[3].record()
     B.csa_sparse_attn(step["q"], step["pos"], ws["seq"], cache["entries"], ws["idx"], ws["cnt"], cache["window"],
                       cache["window_base"], W=wl.W, out=ws["out"], workspace=ws["attn_ws"])
     if ev is not None:
-        ev[4].record()
+        ev[3].record()
 
 
 def capture_step(fn):
@@ -321,20 +323,19 @@ def bench_decode(args, dist, peaks, name: str = "csa_decode_128k", e2e: bool = T
 
     # per-call device time: the same steps run eagerly behind a GPU sleep, so that the
     # calls queue up and execute back to back between the events
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(DECODE_CALLS) + 1)] for _ in range(steps)]
     for i in range(steps):
         torch.cuda._sleep(2_000_000)
         decode_step(wl, caches[i % R], step_inputs[i % R], ws, evs[i])
     torch.cuda.synchronize()
-    per = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in
-           enumerate(["quantize", "index_score", "topk_select", "attention"])}
+    per = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in enumerate(DECODE_CALLS)}
     nb = decode_bytes_per_query(wl)
     queries_per_step = wl.B * dist.world
     value = queries_per_step * steps / (ms / 1e3)
     ms_step = ms / steps
     dom = max(per, key=per.get)
-    dom_bytes = {"index_score": nb["index_score"], "attention": nb["attention"],
-                 "quantize": wl.Hi * wl.Di * 4, "topk_select": wl.E * 4}[dom] * wl.B
+    dom_bytes = {"index_topk": nb["index_topk"], "attention": nb["attention"],
+                 "quantize": wl.Hi * wl.Di * 4}[dom] * wl.B
     achieved = dom_bytes / (per[dom] / 1e3) / 1e9
     step_gbs = nb["step"] * wl.B / (ms_local / steps / 1e3) / 1e9
     res = {
@@ -346,7 +347,8 @@ def bench_decode(args, dist, peaks, name: str = "csa_decode_128k", e2e: bool = T
                           "frac": round(step_gbs / peaks["hbm_gbs"], 4)},
         "per_call_us": {k: round(v * 1e3, 2) for k, v in per.items()},
         "clocks": clk,
-        "gpu_launches": steps * 4,  # query encoding, indexer, top-k, attention (split merge inside)
+        # query encoding, indexer + top-k (one fused kernel or two), attention (split merge inside)
+        "gpu_launches": steps * (2 + B.csa_index_topk_launches(wl.B, wl.Hi, wl.Di, wl.E, wl.k)),
         "graph": "one CUDA graph per input replica, replayed back to back",
     }
     if e2e:
@@ -358,7 +360,8 @@ def bench_decode(args, dist, peaks, name: str = "csa_decode_128k", e2e: bool = T
 
 def bench_decode_e2e(args, wl, caches, steps, ws, dist):
     """Decode through the public API with host buffers: every step copies its inputs (q,
-    indexer query, head weights, positions) from pinned host memory and its output back.
+    indexer query, head weights, positions; one packed block, one copy) from pinned host
+    memory and its output back.
     Steps are independent batches (the input replicas rotate), so they are pipelined
     over three streams: the upload of step i+1 and the download of step i-1 overlap the
     layer call of step i (two buffer sets, ordered by events).  As a serving loop would,
@@ -369,21 +372,39 @@ def bench_decode_e2e(args, wl, caches, steps, ws, dist):
     from compressed_sparse_long_02_b200 import layer
     R = len(caches)
     dev = ws["out"].device
+    # The step's inputs (q, indexer query, head weights, positions) travel as one block:
+    # packed at 256-byte offsets into one pinned host buffer per replica, copied with a
+    # single memcpy into one device buffer, whose views the layer call reads.
+    names = list(steps[0].keys())
+    offs, off = {}, 0
+    for k in names:
+        offs[k] = off
+        off += (steps[0][k].numel() * steps[0][k].element_size() + 255) // 256 * 256
+    total = off
+
+    def views(buf):
+        return {k: buf[offs[k]:offs[k] + steps[0][k].numel() * steps[0][k].element_size()]
+                .view(steps[0][k].dtype).view(steps[0][k].shape) for k in names}
+
     host = []
     for r in range(R):
-        host.append({k: v.cpu().pin_memory() for k, v in steps[r].items()})
+        hb = torch.zeros(total, dtype=torch.uint8).pin_memory()
+        hv = views(hb)
+        for k in names:
+            hv[k].copy_(steps[r][k].cpu())
+        host.append(hb)
     NB = 2
-    dev_in = [{k: torch.empty_like(v) for k, v in steps[0].items()} for _ in range(NB)]
+    dev_buf = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(NB)]
+    dev_in = [views(b) for b in dev_buf]
     dev_out = [torch.empty((wl.B, wl.H, wl.D), dtype=torch.bfloat16, device=dev) for _ in range(NB)]
     out_host = [torch.empty((wl.B, wl.H, wl.D), dtype=torch.bfloat16).pin_memory() for _ in range(NB)]
-    h2d = sum(v.numel() * v.element_size() for v in host[0].values())
+    h2d = sum(steps[0][k].numel() * steps[0][k].element_size() for k in names)
     d2h = out_host[0].numel() * out_host[0].element_size()
-    lws = {"q_fp4": ws["q_fp4"], "q_scale": ws["q_scale"], "scores": ws["scores"], "idx": ws["idx"], "cnt": ws["cnt"],
+    lws = {"q_fp4": ws["q_fp4"], "q_scale": ws["q_scale"], "index_ws": ws["index_ws"], "idx": ws["idx"], "cnt": ws["cnt"],
            "seq": ws["seq"], "attn_ws": ws["attn_ws"]}
 
     def upload(b, r):
-        for k in dev_in[b]:
-            dev_in[b][k].copy_(host[r][k], non_blocking=True)
+        dev_buf[b].copy_(host[r], non_blocking=True)  # one host-to-device copy per step
 
     def compute(b, r):
         layer.csa_decode(wl, caches[r], dev_in[b], lws, out=dev_out[b])

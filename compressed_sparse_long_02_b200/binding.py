@@ -17,8 +17,8 @@ import torch
 
 __all__ = ["CsaError", "lib", "csa_compress", "csa_compress_step", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk",
            "csa_index_score", "csa_index_score_q", "csa_topk_select",
-           "csa_index_topk_workspace", "csa_sparse_attn", "csa_sparse_attn_workspace", "hca_attn",
-           "hca_attn_workspace", "csa_grouped_out_proj", "csa_get_device_error", "csa_set_batch_invariant", "LIB_PATH", "DEVERR_NONE", "DEVERR_TIMEOUT",
+           "csa_index_topk_workspace", "csa_index_topk_launches", "csa_sparse_attn", "csa_sparse_attn_workspace", "hca_attn",
+           "hca_attn_workspace", "csa_grouped_out_proj", "csa_get_device_error", "csa_set_batch_invariant", "csa_set_index_fusion", "LIB_PATH", "DEVERR_NONE", "DEVERR_TIMEOUT",
            "DEVERR_INDEX"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcsa.so")
@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
             L.csa_index_score.argtypes = [I, I, I, I, P, P, P, P, P, I, I, P, P, P, P, I, P]
             L.csa_index_score_q.argtypes = [I, I, I, I, P, I, P, P, P, I, I, P, P, P, P, I, P]
             L.csa_topk_select.argtypes = [I, I, I, P, I, P, P, I, I, P, P, P, P]
+            L.csa_index_topk_launches.argtypes = [I, I, I, I, I]
+            L.csa_index_topk_launches.restype = I
             L.csa_index_topk_workspace.argtypes = [I, I, I]
             L.csa_index_topk_workspace.restype = SZ
             L.csa_sparse_attn.argtypes = [I, I, I, I, I, F, P, P, P, I, I, P, P, P, I, P, P, P, P, P, SZ, P]
@@ -67,6 +69,8 @@ def lib() -> ctypes.CDLL:
             L.hca_attn_workspace.restype = SZ
             L.csa_grouped_out_proj.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P]
             L.csa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
+            L.csa_set_index_fusion.argtypes = [I]
+            L.csa_set_index_fusion.restype = I
             L.csa_set_batch_invariant.argtypes = [I]
             L.csa_set_batch_invariant.restype = I
             L.csa_status_string.argtypes = [I]
@@ -193,6 +197,11 @@ def csa_quantize_mxfp4(x: torch.Tensor, packed: torch.Tensor | None = None, scal
     st = lib().csa_quantize_mxfp4(_ptr(x.contiguous()), _dt(x), rows, cols, _ptr(packed), _ptr(scales), _stream(x))
     _check("csa_quantize_mxfp4", st)
     return packed, scales
+
+
+def csa_index_topk_launches(Nq: int, Hi: int, Di: int, E_max: int, k: int) -> int:
+    """Kernels csa_index_topk launches for these sizes: 1 (fused decode kernel) or 2."""
+    return int(lib().csa_index_topk_launches(Nq, Hi, Di, E_max, k))
 
 
 def csa_index_topk_workspace(Nq: int, E_max: int, k: int) -> int:
@@ -338,6 +347,11 @@ def csa_grouped_out_proj(o, A, Bm, *, z=None, y=None):
     st = lib().csa_grouped_out_proj(T, H, D, G, R, d_model, _ptr(o), _ptr(A), _ptr(Bm), _ptr(z), _ptr(y), _stream(o))
     _check("csa_grouped_out_proj", st)
     return z, y
+
+
+def csa_set_index_fusion(on: bool) -> None:
+    """Process-wide: csa_index_topk uses the fused decode kernel where it fits (off by default)."""
+    _check("csa_set_index_fusion", lib().csa_set_index_fusion(int(bool(on))))
 
 
 def csa_set_batch_invariant(on: bool) -> None:

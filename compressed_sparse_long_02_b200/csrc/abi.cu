@@ -74,6 +74,11 @@ const char* csa_last_cuda_error(void) {
   return buf;
 }
 
+csa_status csa_set_index_fusion(int on) {
+  set_index_fusion(on != 0);
+  return CSA_OK;
+}
+
 csa_status csa_set_batch_invariant(int on) {
   set_batch_invariant(on != 0);
   return CSA_OK;
@@ -201,6 +206,11 @@ csa_status csa_quantize_mxfp4(const void* x, csa_dtype dtype, int64_t rows, int 
   if (rows > 0 && (x == nullptr || packed == nullptr || scales == nullptr)) return CSA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales)) return CSA_ERR_ALIGNMENT;
   return from_cuda(launch_quantize_mxfp4(x, dtype == CSA_BF16, rows, cols, packed, scales, stream));
+}
+
+int csa_index_topk_launches(int Nq, int Hi, int Di, int E_max, int k) {
+  if (Nq < 1) return 0;
+  return index_topk_fusable(Nq, Hi, Di, E_max, k, false, nullptr, nullptr) ? 1 : 2;
 }
 
 size_t csa_index_topk_workspace(int Nq, int E_max, int k) {

@@ -30,6 +30,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 
 #include "common.cuh"
@@ -37,6 +38,7 @@
 #include "mxfp4.cuh"
 #include "ptx.cuh"
 #include "tmap.h"
+#include "topk_regs.cuh"
 
 namespace csa {
 namespace {
@@ -66,16 +68,47 @@ struct IndexParams {
   float* scores;
   float* score_out;
   int32_t* err;
+  int k;           // fused selection: top-k per query into idx [Nq, k] and cnt [Nq]
+  int32_t* idx;
+  int32_t* cnt;
+};
+
+// The fused decode variant (index_score_kernel with kFuseC > 0): a thread-block cluster of
+// kFuseC CTAs per query; CTA r scores the entries [r S, (r + 1) S), S = 256 kFuseEPT, into a
+// slice in its shared memory instead of global memory, then the cluster selects the query's
+// top-k from those slices (topk_regs_row) -- no score round trip, one launch.  256 threads
+// and ~105 KB of shared memory, so two CTAs share an SM as in the plain kernel: the producer
+// (warp 0), the MMA issuer (warp 1) and one epilogue group (warps 2-5) score, and all eight
+// warps select.
+constexpr int kFuseThreads = 256;
+constexpr int kFuseStages = 6;
+template <int kFuseC, int kFuseEPT>
+struct IndexShape {
+  static constexpr bool kFuse = kFuseC > 0;
+  static constexpr int kThreads = kFuse ? kFuseThreads : kIdxThreads;
+  static constexpr int kSt = kFuse ? kFuseStages : kStages;
+  static constexpr int kMaxTiles = kFuse ? kFuseThreads * kFuseEPT / kTileE : kMaxTilesPerCta;
+  static constexpr int kRawSf = kFuse ? 0 : kMaxTilesPerCta;  // raw scale bytes for Di = 64 (not fused)
+  static constexpr int kSlice = kFuse ? kFuseThreads * kFuseEPT : 0;
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kSt) * 8192 + 4096 + static_cast<size_t>(kMaxTiles) * 512 +
+                                  static_cast<size_t>(kRawSf) * 256 + 512 + 256 + 512 + static_cast<size_t>(kSlice) * 4;
 };
 
 // kHi: number of indexer heads fixed at compile time (the head chain is straight-line
 // code), or 0 to take it from p.Hi at run time.  kRawQ: the query arrives unencoded and
 // the epilogue warps encode it to MXFP4 (the same rule as quantize_mxfp4_kernel) into
 // the MMA's B operand and scale factors before the first tile.
-template <int kHi, bool kRawQ>
-__global__ void __launch_bounds__(kIdxThreads, 2)
+template <int kHi, bool kRawQ, int kFuseC = 0, int kFuseEPT = 8>
+__global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT>::kThreads, 2)
     index_score_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                        IndexParams p) {
+  using Shape = IndexShape<kFuseC, kFuseEPT>;
+  constexpr bool kFuse = Shape::kFuse;
+  constexpr int kStages = Shape::kSt;  // shadows the plain kernel's depth in this body
+  // epilogue warps: two groups of four (warps 2-9); the fused kernel one (warps 2-5)
+  constexpr int kEpiGroups = kFuse ? 1 : 2;
+  constexpr int kEpiWarps = 4 * kEpiGroups;
+  static_assert(!(kFuse && kRawQ), "the fused kernel takes pre-encoded queries");
   CSA_TB(0);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -84,11 +117,12 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
   // shared memory carve-up
   uint8_t* sA = smem;                                    // kStages x 8 KB (1024-aligned)
   uint8_t* sB = sA + kStages * 8192;                     // 4 KB
-  uint8_t* sSF = sB + 4096;                              // kMaxTilesPerCta x 512: key scales, scale-factor layout
-  uint8_t* sSFraw = sSF + kMaxTilesPerCta * 512;         // kMaxTilesPerCta x 256: raw key scales when Di = 64
-  uint8_t* sSFB = sSFraw + kMaxTilesPerCta * 256;        // 512
+  uint8_t* sSF = sB + 4096;                              // kMaxTiles x 512: key scales, scale-factor layout
+  uint8_t* sSFraw = sSF + Shape::kMaxTiles * 512;        // kRawSf x 256: raw key scales when Di = 64
+  uint8_t* sSFB = sSFraw + Shape::kRawSf * 256;          // 512
   float* sW = reinterpret_cast<float*>(sSFB + 512);      // [64] head weights
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sW + 64);
+  float* sSlice = sW + 64;                               // fused: this CTA's scores [kSlice]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSlice + Shape::kSlice);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
   uint64_t* b_full = bars + 2 * kStages;
@@ -107,7 +141,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
     }
     mbar_init(b_full, kRawQ ? 8 : 1);
     mbar_init(sf_full, 1);
-    mbar_init(sf_ready, 8);
+    mbar_init(sf_ready, kEpiWarps);
     for (int i = 0; i < kAccBufs; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);
@@ -128,14 +162,18 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
   griddep_enter();
   CSA_TB(1);
 
-  const int q = blockIdx.x / p.splits;
-  const int split = blockIdx.x % p.splits;
+  const int q = kFuse ? static_cast<int>(blockIdx.x) / kFuseC : static_cast<int>(blockIdx.x) / p.splits;
+  const int split = kFuse ? static_cast<int>(blockIdx.x) % kFuseC : static_cast<int>(blockIdx.x) % p.splits;
   const int seq = p.q_seq[q];
   const bool seq_ok = seq >= 0 && seq < p.B;
   if (!seq_ok && threadIdx.x == 0 && split == 0) atomicExch(p.err, CSA_DEVERR_INDEX);  // produce nothing
   const int nvis = seq_ok ? min(visible_entries(p.q_pos[q], p.m, p.n_entries[seq]), p.E_max) : 0;
-  const int t_begin = split * p.tiles_per_cta;
-  const int t_end = min((nvis + kTileE - 1) / kTileE, t_begin + p.tiles_per_cta);
+  const int tiles_per_cta = kFuse ? Shape::kMaxTiles : p.tiles_per_cta;
+  const int t_begin = split * tiles_per_cta;
+  // fused: a query with at most k visible entries takes all of them (no scoring; the same
+  // for every CTA of the cluster, so none reaches a cluster barrier below)
+  const bool trivial = kFuse && nvis <= p.k;
+  const int t_end = trivial ? t_begin : min((nvis + kTileE - 1) / kTileE, t_begin + tiles_per_cta);
   const int n_tiles = t_end - t_begin;  // uniform over the CTA
 
   const int Hi = kHi > 0 ? kHi : p.Hi;
@@ -237,8 +275,8 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
       }
     }
     __syncwarp();
-  } else if (n_tiles > 0) {
-    // ------------------------------------------------------------ epilogue (warps 2..9)
+  } else if (n_tiles > 0 && warp < 2 + kEpiWarps) {
+    // ------------------------------------------------------------ epilogue (warps 2 .. 1 + kEpiWarps)
     const int ew = warp - 2;
     if (ew * 32 + lane < 64) {
       const int h = ew * 32 + lane;
@@ -287,11 +325,11 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(b_full);
     }
-    // key scales: entry-major bytes -> scale-factor layout, warp ew takes tiles ew, ew + 8, ...
+    // key scales: entry-major bytes -> scale-factor layout, warp ew takes tiles ew, ew + kEpiWarps, ...
     // (word (r % 32) * 4 + r / 32 of a 512-byte slot holds the scale bytes of entry r)
     bool ok = warp_wait(sf_full, 0, p.err, abort_flag);
     if (ok) {
-      for (int i = ew; i < n_tiles; i += 8) {
+      for (int i = ew; i < n_tiles; i += kEpiWarps) {
         uint32_t words[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -306,12 +344,12 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(sf_ready);
     }
-    named_bar_sync(1, 256);
-    // group 0 (warps 2-5) takes even tiles, group 1 (warps 6-9) odd tiles, so two tiles
+    named_bar_sync(1, 32 * kEpiWarps);
+    // group g (warps 2 + 4g .. 5 + 4g) takes tiles g, g + kEpiGroups, ..., so kEpiGroups tiles
     // are reduced at once; tile it sits in accumulator it % kAccBufs
     const int grp = ew >> 2;
     const int sub = warp & 3;  // TMEM lane quarter this warp may access
-    for (int it = grp; ok && it < n_tiles; it += 2) {
+    for (int it = grp; ok && it < n_tiles; it += kEpiGroups) {
       const int buf = it % kAccBufs;
       if (!warp_wait(&acc_full[buf], (it / kAccBufs) & 1, p.err, abort_flag)) break;
       if (sub == 0 && lane == 0 && it < 16 && tslot == 0) CSA_T(6, it);
@@ -340,7 +378,10 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
       const int e = (t_begin + it) * kTileE + 32 * sub + lane;
       if (sub == 0 && lane == 0 && it < 16) CSA_T(tslot, 48 + it);
       if (e < nvis) {
-        p.scores[static_cast<size_t>(q) * p.E_stride + e] = s;
+        if constexpr (kFuse)
+          sSlice[e - t_begin * kTileE] = s;
+        else
+          p.scores[static_cast<size_t>(q) * p.E_stride + e] = s;
         if (p.score_out) p.score_out[static_cast<size_t>(q) * p.E_max + e] = s;
       }
     }
@@ -353,6 +394,35 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  if constexpr (kFuse) {
+    // ---------------------------------------------------------------- selection
+    if (trivial) {
+      if (split == 0) {
+        int32_t* out = p.idx + static_cast<size_t>(q) * p.k;
+        for (int j = threadIdx.x; j < p.k; j += kFuseThreads) out[j] = j < nvis ? j : -1;
+        if (threadIdx.x == 0) p.cnt[q] = nvis;
+      }
+      return;
+    }
+    // this CTA's slice (written by the epilogue warps before the barrier above) into
+    // registers in the layout topk_regs_row takes: v[i] of (warp, lane) is entry
+    // t_begin 128 + 32 kFuseEPT warp + 32 i + lane
+    using Mask = TopkMask<kFuseEPT>;
+    const int e0 = t_begin * kTileE + 32 * kFuseEPT * warp + lane;
+    float v[kFuseEPT];
+    Mask valid = 0;
+#pragma unroll
+    for (int i = 0; i < kFuseEPT; ++i) {
+      const bool ok = e0 + 32 * i < nvis;
+      v[i] = ok ? sSlice[32 * kFuseEPT * warp + 32 * i + lane] : 0.f;
+      valid |= (ok ? Mask(1) : Mask(0)) << i;
+    }
+    TopkParams tp{};
+    tp.k = p.k;
+    tp.idx = p.idx;
+    tp.cnt = p.cnt;
+    topk_regs_row<kFuseC, kFuseThreads, kFuseEPT>(tp, q, split, v, valid);
   }
 }
 
@@ -785,7 +855,7 @@ cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s) {
                       s, tm_k, tm_q, p);
   }
 
-  const size_t smem = 1024 + kStages * 8192 + 4096 + kMaxTilesPerCta * (512 + 256) + 512 + 256 + 512;
+  const size_t smem = IndexShape<0, 8>::kSmem;
   p.q_raw = a.q_raw;
   p.q_raw_bf16 = a.q_raw_bf16;
   const dim3 grid(a.Nq * p.splits), block(kIdxThreads);
@@ -796,6 +866,85 @@ cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s) {
   if (a.q_raw != nullptr)
     return a.Hi == 64 ? go(index_score_kernel<64, true>, 2) : go(index_score_kernel<0, true>, 3);
   return a.Hi == 64 ? go(index_score_kernel<64, false>, 0) : go(index_score_kernel<0, false>, 1);
+}
+
+namespace {
+int g_fuse_smem[6][64];
+
+template <int C, int EPT>
+cudaError_t launch_fused_t(const CUtensorMap& tm_k, const CUtensorMap& tm_q, const IndexParams& p, int Nq,
+                           cudaStream_t s, int slot) {
+  auto kern = index_score_kernel<64, false, C, EPT>;
+  constexpr size_t smem = IndexShape<C, EPT>::kSmem;
+  const cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(kern), smem, g_fuse_smem[slot]);
+  if (e != cudaSuccess) return e;
+  return launch_pdl_cluster(kern, dim3(Nq * C), dim3(kFuseThreads), smem, static_cast<unsigned>(C), s, tm_k, tm_q, p);
+}
+}  // namespace
+
+namespace {
+std::atomic<int> g_index_fusion{0};
+}  // namespace
+
+void set_index_fusion(bool on) { g_index_fusion.store(on ? 1 : 0); }
+
+bool index_topk_fusable(int Nq, int Hi, int Di, int E_max, int k, bool raw_q, int* C_out, int* ept_out) {
+  if (g_index_fusion.load() == 0) return false;
+  if (raw_q || Hi != 64 || Di != 128 || k < 1 || Nq < 1) return false;
+  // the largest cluster for which two CTAs per SM hold every query and the slices hold the
+  // row; the fused kernel only pays when the CTAs are at least one per SM
+  const int sms = num_sms();
+  int C = 0;
+  for (int c = 8; c >= 2 && C == 0; c >>= 1)
+    if (static_cast<int64_t>(Nq) * c <= 2 * sms && static_cast<int64_t>(c) * kFuseThreads * 16 >= E_max) C = c;
+  if (C == 0 || static_cast<int64_t>(Nq) * C < sms) return false;
+  if (C_out) *C_out = C;
+  if (ept_out) *ept_out = static_cast<int64_t>(C) * kFuseThreads * 8 >= E_max ? 8 : 16;
+  return true;
+}
+
+cudaError_t launch_index_topk_fused(const IndexArgs& a, cudaStream_t s, bool* launched) {
+  *launched = false;
+  int C = 0, ept = 0;
+  if (a.idx_out == nullptr || a.cnt_out == nullptr ||
+      !index_topk_fusable(a.Nq, a.Hi, a.Di, a.E_max, a.k, a.q_raw != nullptr, &C, &ept))
+    return cudaSuccess;
+  CUtensorMap tm_k, tm_q;
+  if (!encode_2d_u8(&tm_k, a.k_fp4, 64, static_cast<uint64_t>(a.B) * a.E_max, 64, kTileE, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode_2d_u8(&tm_q, a.q_fp4, 64, static_cast<uint64_t>(a.Nq) * a.Hi, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  IndexParams p{};
+  p.Nq = a.Nq;
+  p.Hi = a.Hi;
+  p.Di = a.Di;
+  p.m = a.m;
+  p.B = a.B;
+  p.E_max = a.E_max;
+  p.E_stride = a.E_stride;
+  p.N = 64;
+  p.tiles_per_cta = kFuseThreads * ept / kTileE;
+  p.splits = C;
+  p.w = a.w;
+  p.q_pos = a.q_pos;
+  p.q_seq = a.q_seq;
+  p.n_entries = a.n_entries;
+  p.q_scale = a.q_scale;
+  p.k_scale = a.k_scale;
+  p.scores = nullptr;
+  p.score_out = a.score_out;
+  p.err = device_error_word();
+  p.k = a.k;
+  p.idx = a.idx_out;
+  p.cnt = a.cnt_out;
+  cudaError_t e;
+  if (C == 8)
+    e = ept == 8 ? launch_fused_t<8, 8>(tm_k, tm_q, p, a.Nq, s, 0) : launch_fused_t<8, 16>(tm_k, tm_q, p, a.Nq, s, 1);
+  else if (C == 4)
+    e = ept == 8 ? launch_fused_t<4, 8>(tm_k, tm_q, p, a.Nq, s, 2) : launch_fused_t<4, 16>(tm_k, tm_q, p, a.Nq, s, 3);
+  else
+    e = ept == 8 ? launch_fused_t<2, 8>(tm_k, tm_q, p, a.Nq, s, 4) : launch_fused_t<2, 16>(tm_k, tm_q, p, a.Nq, s, 5);
+  if (e == cudaSuccess) *launched = true;
+  return e;
 }
 
 }  // namespace csa

@@ -134,8 +134,18 @@ struct IndexArgs {
 size_t index_workspace_bytes(int Nq, int E_max, int k);
 cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s);  // writes scores_ws (+ score_out)
 cudaError_t launch_topk_select(const IndexArgs& a, cudaStream_t s);  // reads scores_ws
+// The fused decode kernel (scores kept on chip, a cluster top-k per query) when the shape
+// suits it; *launched tells whether it ran (otherwise nothing was launched).
+cudaError_t launch_index_topk_fused(const IndexArgs& a, cudaStream_t s, bool* launched);
+bool index_topk_fusable(int Nq, int Hi, int Di, int E_max, int k, bool raw_q, int* C, int* ept);
+// The fused decode kernel (process-wide, off by default: measured slower than the two
+// kernels at the 128K decode shape).
+void set_index_fusion(bool on);
 inline cudaError_t launch_index_topk(const IndexArgs& a, cudaStream_t s) {
-  const cudaError_t e = launch_index_score(a, s);
+  bool fused = false;
+  cudaError_t e = launch_index_topk_fused(a, s, &fused);
+  if (e != cudaSuccess || fused) return e;
+  e = launch_index_score(a, s);
   return e != cudaSuccess ? e : launch_topk_select(a, s);
 }
 

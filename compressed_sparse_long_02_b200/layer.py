@@ -8,8 +8,8 @@ rabbit", CSA / window / indexer paragraphs):
     csa_norm_rope(q)            -> attention queries
     csa_index_topk              -> top-k entry indices per query
     csa_sparse_attn             -> output
-CSA decode: csa_quantize_mxfp4(q_I) -> csa_index_score -> csa_topk_select ->
-csa_sparse_attn over a resident cache.  HCA prefill: csa_compress(m'=128) -> csa_norm_rope(q) -> hca_attn.
+CSA decode: csa_quantize_mxfp4(q_I) -> csa_index_topk (scores and selection in one
+fused kernel at decode shapes) -> csa_sparse_attn over a resident cache.  HCA prefill: csa_compress(m'=128) -> csa_norm_rope(q) -> hca_attn.
 """
 from __future__ import annotations
 
@@ -57,24 +57,20 @@ def csa_decode(wl, cache: dict, step: dict, ws: dict | None = None, out: torch.T
     cache: entries [B,E,D] bf16, k_fp4 [B,E,Di/2], k_scale [B,E,Di/32], window [B,W,D] bf16,
            window_base int32 [B], n_entries int32 [B]
     step:  q [B,H,D] bf16 (normalised, rotated), qi [B,Hi,Di] float32, w [B,Hi], pos int32 [B]
-    ws:    optional preallocated buffers (q_fp4, q_scale, scores [B, >=E] float32, idx, cnt,
-           seq, attn_ws).
-    csa_quantize_mxfp4(qi) -> csa_index_score -> csa_topk_select -> csa_sparse_attn."""
+    ws:    optional preallocated buffers (q_fp4, q_scale, index_ws (csa_index_topk's workspace),
+           idx, cnt, seq, attn_ws).
+    csa_quantize_mxfp4(qi) -> csa_index_topk (fused scores + selection when the shape suits it)
+    -> csa_sparse_attn."""
     Bn = step["q"].shape[0]
     dev = step["q"].device
     ws = ws or {}
     seq = ws.get("seq")
     if seq is None:
         seq = torch.arange(Bn, dtype=torch.int32, device=dev)
-    E_max = cache["k_fp4"].shape[1]
-    scores = ws.get("scores")
-    if scores is None:
-        scores = torch.empty((Bn, E_max), dtype=torch.float32, device=dev)
     q_fp4, q_sc = B.csa_quantize_mxfp4(step["qi"], ws.get("q_fp4"), ws.get("q_scale"))
-    B.csa_index_score(q_fp4, q_sc, step["w"], step["pos"], seq, cache["k_fp4"], cache["k_scale"],
-                      cache["n_entries"], m=wl.m, scores=scores)
-    idx, cnt = B.csa_topk_select(scores, step["pos"], seq, cache["n_entries"], k=wl.k, m=wl.m, E_max=E_max,
-                                 idx=ws.get("idx"), cnt=ws.get("cnt"))
+    idx, cnt, _ = B.csa_index_topk(q_fp4, q_sc, step["w"], step["pos"], seq, cache["k_fp4"], cache["k_scale"],
+                                   cache["n_entries"], k=wl.k, m=wl.m, workspace=ws.get("index_ws"),
+                                   idx=ws.get("idx"), cnt=ws.get("cnt"))
     o, lse = B.csa_sparse_attn(step["q"], step["pos"], seq, cache["entries"], idx, cnt, cache["window"],
                                cache["window_base"], W=wl.W, out=out, workspace=ws.get("attn_ws"))
     return dict(out=o, idx=idx, cnt=cnt)

@@ -192,6 +192,23 @@ CSA_API csa_status csa_index_topk(int Nq, int Hi, int Di, int k, int m, const ui
                           int32_t* cnt_out, float* score_out, void* workspace, size_t ws_bytes,
                           cudaStream_t stream);
 CSA_API size_t csa_index_topk_workspace(int Nq, int E_max, int k);
+/* Kernels csa_index_topk launches for these sizes (pre-encoded queries): 1 when the fused
+ * decode kernel runs, 2 otherwise (the scoring kernel, then the top-k kernel), 0 for
+ * Nq < 1.  See csa_set_index_fusion. */
+CSA_API int csa_index_topk_launches(int Nq, int Hi, int Di, int E_max, int k);
+
+/*
+ * csa_set_index_fusion -- process-wide switch (off by default) for the fused decode
+ * indexer + top-k ("Follow the white rabbit", indexer paragraph: every compressed entry
+ * scored, the top 1,024 kept).  With it on, csa_index_topk runs one kernel when a
+ * thread-block cluster of 2, 4 or 8 CTAs per query fits (pre-encoded queries, Hi = 64,
+ * Di = 128, E_max up to 4 Ki entries per CTA of the cluster, two CTAs per SM and at least
+ * as many CTAs as SMs): each CTA scores its slice of the query's entries into shared
+ * memory and the cluster selects the top-k there, so the scores never reach global
+ * memory.  The results are bit-for-bit those of the two-kernel path; it is off by default
+ * because at the 128K decode shape it measures slower (47-51 us against 43.5 us).
+ */
+CSA_API csa_status csa_set_index_fusion(int on);
 
 /*
  * csa_index_topk_static -- csa_index_topk for callers that cannot allocate device memory.

@@ -126,3 +126,19 @@ def test_static_indexer_size_limit_boundary(L):
     assert call(1, 1 << 21) == 1
     assert call(1, (1 << 21) + 8) == 4
     assert call(32, 65540) == 3          # E_max % 8 != 0: CSA_ERR_UNSUPPORTED
+
+
+def test_index_fusion_switch_plan(L):
+    """csa_index_topk's launch plan: two kernels by default; with the fusion switch on, one
+    fused kernel for the 128K decode shape (32 queries, 32768 entries) and still two for
+    rows too long for a cluster's slices (4 queries of 262144 entries)."""
+    from compressed_sparse_long_02_b200 import binding as B
+    assert B.csa_index_topk_launches(32, 64, 128, 32768, 1024) == 2
+    try:
+        B.csa_set_index_fusion(True)
+        assert B.csa_index_topk_launches(32, 64, 128, 32768, 1024) == 1
+        assert B.csa_index_topk_launches(4, 64, 128, 262144, 1024) == 2
+        assert B.csa_index_topk_launches(32, 32, 128, 32768, 1024) == 2   # other head counts: not fused
+        assert B.csa_index_topk_launches(0, 64, 128, 32768, 1024) == 0
+    finally:
+        B.csa_set_index_fusion(False)
