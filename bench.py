@@ -358,6 +358,98 @@ def bench_decode(args, dist, peaks, name: str = "csa_decode_128k", e2e: bool = T
     return wl, res
 
 
+def bench_decode_mq(args, dist, peaks, name: str = "csa_decode_128k", steps: int = 20):
+    """Multi-query decode at the 128K shape: every sequence advances by two tokens per
+    step (a new token and one draft, at positions L-2 and L-1 of the resident cache), so a
+    step has 2 x B queries.  The indexer runs grouped (csa_index_topk_grouped: the two
+    queries of a sequence read its key cache once) and, for comparison, ungrouped on the
+    same inputs; attention is per query either way.  Graph replays, input replicas
+    rotating as in the headline line."""
+    import torch
+    from compressed_sparse_long_02_b200 import binding as B
+    from compressed_sparse_long_02_b200 import synth
+    wl = synth.WORKLOADS[name]
+    dev = torch.device("cuda", dist.local_rank)
+    R = args.replicas
+    caches, _, _ = setup_decode(wl, dev, R)
+    Bn, nq = wl.B, 2 * wl.B
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.seed * 104729)
+    L = wl.E * wl.m
+    steps_in = []
+    for _ in range(R):
+        steps_in.append({
+            "q": torch.randn((nq, wl.H, wl.D), generator=g, device=dev).to(torch.bfloat16),
+            "qi": torch.randn((nq, wl.Hi, wl.Di), generator=g, device=dev),
+            "w": torch.rand((nq, wl.Hi), generator=g, device=dev),
+            "pos": torch.tensor([L - 2, L - 1] * Bn, dtype=torch.int32, device=dev)})
+    ws = {
+        "index_ws": torch.empty(B.csa_index_topk_workspace(nq, wl.E, wl.k), dtype=torch.uint8, device=dev),
+        "idx": torch.empty((nq, wl.k), dtype=torch.int32, device=dev),
+        "cnt": torch.empty((nq,), dtype=torch.int32, device=dev),
+        "seq": torch.arange(Bn, dtype=torch.int32, device=dev).repeat_interleave(2),
+        "attn_ws": torch.empty(B.csa_sparse_attn_workspace(nq, wl.H, wl.D, wl.k, wl.W), dtype=torch.uint8,
+                               device=dev),
+        "out": torch.empty((nq, wl.H, wl.D), dtype=torch.bfloat16, device=dev),
+        "q_fp4": torch.empty((nq, wl.Hi, wl.Di // 2), dtype=torch.uint8, device=dev),
+        "q_scale": torch.empty((nq, wl.Hi, wl.Di // 32), dtype=torch.uint8, device=dev)}
+
+    def step(i, q_group, ev=None):
+        c, st = caches[i % R], steps_in[i % R]
+        if ev is not None:
+            ev[0].record()
+        B.csa_quantize_mxfp4(st["qi"], ws["q_fp4"], ws["q_scale"])
+        if ev is not None:
+            ev[1].record()
+        B.csa_index_topk(ws["q_fp4"], ws["q_scale"], st["w"], st["pos"], ws["seq"], c["k_fp4"], c["k_scale"],
+                         c["n_entries"], k=wl.k, m=wl.m, workspace=ws["index_ws"], idx=ws["idx"], cnt=ws["cnt"],
+                         q_group=q_group)
+        if ev is not None:
+            ev[2].record()
+        B.csa_sparse_attn(st["q"], st["pos"], ws["seq"], c["entries"], ws["idx"], ws["cnt"], c["window"],
+                          c["window_base"], W=wl.W, out=ws["out"], workspace=ws["attn_ws"])
+        if ev is not None:
+            ev[3].record()
+
+    out = {"workload": name + "_2tok", "sequences": Bn, "queries_per_step": nq, "unit": UNIT}
+    for q_group in (2, 1):
+        for i in range(R):
+            step(i, q_group)
+        torch.cuda.synchronize()
+        graphs = [capture_step(lambda i=i: step(i, q_group)) for i in range(R)]
+        for i in range(args.warmup):
+            graphs[i % R].replay()
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        s0.record()
+        for i in range(steps):
+            graphs[i % R].replay()
+        s1.record()
+        torch.cuda.synchronize()
+        ms = dist.max(s0.elapsed_time(s1)) / steps
+        assert B.csa_get_device_error() == 0
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        for i in range(steps):
+            torch.cuda._sleep(2_000_000)
+            step(i, q_group, evs[i])
+        torch.cuda.synchronize()
+        per = {n: round(1e3 * statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs), 2)
+               for j, n in enumerate(DECODE_CALLS)}
+        key = "grouped" if q_group == 2 else "ungrouped"
+        out[key] = {"value": nq * dist.world / (ms / 1e3), "ms_per_step": ms, "per_call_us": per}
+        del graphs
+    # the grouped indexer reads each sequence's keys once: its HBM roofline
+    keys = wl.E * (wl.Di // 2 + wl.Di // 32) * Bn
+    us = out["grouped"]["per_call_us"]["index_topk"]
+    out["index_topk_roofline"] = {"bound": "hbm", "algorithmic_bytes": keys, "achieved": round(keys / us / 1e3, 1),
+                                  "unit": "GB/s", "frac": round(keys / us / 1e3 / peaks["hbm_gbs"], 4)}
+    out["value"] = out["grouped"]["value"]
+    del caches, steps_in, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_decode_e2e(args, wl, caches, steps, ws, dist):
     """Decode through the public API with host buffers: every step copies its inputs (q,
     indexer query, head weights, positions; one packed block, one copy) from pinned host
@@ -496,8 +588,8 @@ def prefill_calls(wl, t, dev):
                 want_fp4=True, E_max=E_pad))),
             ("quantize_qi", lambda: st.__setitem__("qq", B.csa_quantize_mxfp4(t["qi"][0]))),
         ]
-    calls.append(("norm_rope_q", lambda: st.__setitem__("q", B.csa_norm_rope(
-        t["q"][0], pos, norm=wl.norm, eps=wl.eps, rope_dims=wl.rope_dims, theta=wl.theta))))
+    q = t["q"][0]  # raw queries: the attention call applies their RMSNorm + RoPE as it loads them
+    prep = dict(norm=wl.norm, eps=wl.eps, rope_dims=wl.rope_dims, theta=wl.theta)
     if wl.kind == "csa_prefill":
         w = t["w"][0].contiguous()
         scores = torch.empty((T, max(8, (E + 7) // 8 * 8)), dtype=torch.float32, device=dev)  # no fill inside the timing
@@ -508,12 +600,12 @@ def prefill_calls(wl, t, dev):
             ("topk_select", lambda: st.__setitem__("sel", B.csa_topk_select(
                 st["scores"], pos, seq, ne, k=wl.k, m=wl.m, E_max=st["keys"]["fp4"].shape[1]))),
             ("attention", lambda: st.__setitem__("out", B.csa_sparse_attn(
-                st["q"], pos, seq, st["pool"]["entries"], st["sel"][0], st["sel"][1], st["pool"]["window"], zero,
-                W=wl.W)[0])),
+                q, pos, seq, st["pool"]["entries"], st["sel"][0], st["sel"][1], st["pool"]["window"], zero,
+                W=wl.W, prep=prep)[0])),
         ]
     else:
         calls.append(("attention", lambda: st.__setitem__("out", B.hca_attn(
-            st["q"], pos, seq, st["pool"]["entries"], ne, st["pool"]["window"], zero, mprime=wl.m, W=wl.W)[0])))
+            q, pos, seq, st["pool"]["entries"], ne, st["pool"]["window"], zero, mprime=wl.m, W=wl.W, prep=prep)[0])))
     return calls
 
 
@@ -521,9 +613,8 @@ def prefill_work(wl) -> dict:
     """Algorithmic work of each prefill call: (bound, amount, unit) with bytes for the
     HBM-bound calls (compulsory traffic: inputs read once, outputs written once) and
     dense FLOPs for the contractions."""
-    T, C, E, H, s = wl.T, wl.C, wl.E, wl.H, (2 if wl.dtype == "bf16" else 4)
-    w = {"compress_kv": ("hbm", 2 * T * C * s + E * C * 2 + T * C * 2),  # kv, z in; entries, window rows out
-         "norm_rope_q": ("hbm", T * H * C * (s + 2))}
+    T, C, E, s = wl.T, wl.C, wl.E, (2 if wl.dtype == "bf16" else 4)
+    w = {"compress_kv": ("hbm", 2 * T * C * s + E * C * 2 + T * C * 2)}  # kv, z in; entries, window rows out
     if wl.kind == "csa_prefill":
         Hi, Di = wl.Hi, wl.Di
         vis = sum(min((t + 1) // wl.m, E) for t in range(T))
@@ -797,6 +888,7 @@ def main():
                                  "step_roofline": r1["step_roofline"], "roofline": r1["roofline"],
                                  "per_call_us": r1["per_call_us"], "clocks": r1["clocks"]}
             line["gpu_launches_decode_1m"] = r1["gpu_launches"]
+            line["decode_2tok"] = bench_decode_mq(args, dist, peaks)
             line["prefill"] = bench_prefill("csa_prefill_8k", 5, 2, dist, peaks, tp)
             line["hca_prefill"] = bench_prefill("hca_prefill_64k", 3, 1, dist, peaks, tp)
             line["out_proj"] = bench_out_proj(dist, peaks)

@@ -18,6 +18,7 @@ import torch
 __all__ = ["CsaError", "lib", "csa_compress", "csa_compress_step", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk",
            "csa_index_score", "csa_index_score_q", "csa_topk_select",
            "csa_index_topk_workspace", "csa_index_topk_launches", "csa_sparse_attn", "csa_sparse_attn_workspace", "hca_attn",
+           "csa_sparse_attn_ex", "hca_attn_ex", "csa_index_topk_grouped",
            "hca_attn_workspace", "csa_grouped_out_proj", "csa_get_device_error", "csa_set_batch_invariant", "csa_set_index_fusion", "LIB_PATH", "DEVERR_NONE", "DEVERR_TIMEOUT",
            "DEVERR_INDEX"]
 
@@ -32,6 +33,19 @@ class CsaError(RuntimeError):
     def __init__(self, fn: str, status: int, msg: str):
         super().__init__(f"{fn}: status {status} ({msg})")
         self.status = status
+
+
+class _QPrep(ctypes.Structure):
+    _fields_ = [("norm", ctypes.c_int), ("eps", ctypes.c_float), ("rope_dims", ctypes.c_int),
+                ("rope_theta", ctypes.c_float)]
+
+
+def _q_prep(prep: dict | None):
+    """csa_q_prep from dict(norm=..., eps=..., rope_dims=..., theta=...), or NULL."""
+    if prep is None:
+        return None
+    return ctypes.byref(_QPrep(int(bool(prep.get("norm", True))), float(prep.get("eps", 1e-6)),
+                               int(prep.get("rope_dims", 0)), float(prep.get("theta", 10000.0))))
 
 
 class _PoolCfg(ctypes.Structure):
@@ -57,6 +71,7 @@ def lib() -> ctypes.CDLL:
             L.csa_index_score.argtypes = [I, I, I, I, P, P, P, P, P, I, I, P, P, P, P, I, P]
             L.csa_index_score_q.argtypes = [I, I, I, I, P, I, P, P, P, I, I, P, P, P, P, I, P]
             L.csa_topk_select.argtypes = [I, I, I, P, I, P, P, I, I, P, P, P, P]
+            L.csa_index_topk_grouped.argtypes = [I] + L.csa_index_topk.argtypes
             L.csa_index_topk_launches.argtypes = [I, I, I, I, I]
             L.csa_index_topk_launches.restype = I
             L.csa_index_topk_workspace.argtypes = [I, I, I]
@@ -65,6 +80,8 @@ def lib() -> ctypes.CDLL:
             L.csa_sparse_attn_workspace.argtypes = [I, I, I, I, I]
             L.csa_sparse_attn_workspace.restype = SZ
             L.hca_attn.argtypes = [I, I, I, I, I, F, P, P, P, I, I, P, P, I, P, P, P, P, P, SZ, P]
+            L.csa_sparse_attn_ex.argtypes = [ctypes.POINTER(_QPrep)] + L.csa_sparse_attn.argtypes
+            L.hca_attn_ex.argtypes = [ctypes.POINTER(_QPrep)] + L.hca_attn.argtypes
             L.hca_attn_workspace.argtypes = [I, I, I, I, I]
             L.hca_attn_workspace.restype = SZ
             L.csa_grouped_out_proj.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P]
@@ -80,7 +97,8 @@ def lib() -> ctypes.CDLL:
             for fn in ("csa_compress", "csa_compress_step", "csa_norm_rope", "csa_quantize_mxfp4", "csa_index_topk", "csa_index_score",
                        "csa_index_score_q",
                        "csa_topk_select", "csa_sparse_attn",
-                       "hca_attn", "csa_grouped_out_proj", "csa_get_device_error"):
+                       "hca_attn", "csa_sparse_attn_ex", "hca_attn_ex", "csa_grouped_out_proj", "csa_index_topk_grouped",
+                       "csa_get_device_error"):
                 getattr(L, fn).restype = I
             _lib = L
     return _lib
@@ -209,8 +227,11 @@ def csa_index_topk_workspace(Nq: int, E_max: int, k: int) -> int:
 
 
 def csa_index_topk(q_fp4, q_scale, w, q_pos, q_seq, k_fp4, k_scale, n_entries, *, k: int, m: int,
-                   want_scores: bool = False, workspace: torch.Tensor | None = None, idx=None, cnt=None):
-    """Lightning-indexer scores + top-k.  Returns (idx [Nq,k] int32, cnt [Nq] int32, scores or None)."""
+                   want_scores: bool = False, workspace: torch.Tensor | None = None, idx=None, cnt=None,
+                   q_group: int = 1):
+    """Lightning-indexer scores + top-k.  Returns (idx [Nq,k] int32, cnt [Nq] int32, scores or None).
+    q_group = 2: rows 2g and 2g+1 name one sequence and share its key reads
+    (csa_index_topk_grouped)."""
     Nq, Hi, half = q_fp4.shape
     Di = half * 2
     B, E_max, _ = k_fp4.shape
@@ -228,11 +249,16 @@ def csa_index_topk(q_fp4, q_scale, w, q_pos, q_seq, k_fp4, k_scale, n_entries, *
     need = csa_index_topk_workspace(Nq, E_max, k)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    st = lib().csa_index_topk(Nq, Hi, Di, k, m, _ptr(q_fp4), _ptr(q_scale), _ptr(w), _ptr(q_pos), _ptr(q_seq), B,
-                              E_max, _ptr(k_fp4), _ptr(k_scale), _ptr(n_entries), _ptr(idx), _ptr(cnt),
-                              _ptr(scores), _ptr(workspace), workspace.numel(), _stream(q_fp4))
+    st = lib().csa_index_topk_grouped(q_group, Nq, Hi, Di, k, m, _ptr(q_fp4), _ptr(q_scale), _ptr(w), _ptr(q_pos),
+                                      _ptr(q_seq), B, E_max, _ptr(k_fp4), _ptr(k_scale), _ptr(n_entries), _ptr(idx),
+                                      _ptr(cnt), _ptr(scores), _ptr(workspace), workspace.numel(), _stream(q_fp4))
     _check("csa_index_topk", st)
     return idx, cnt, scores
+
+
+def csa_index_topk_grouped(q_group: int, *args, **kw):
+    """csa_index_topk with rows in groups of q_group sharing a sequence (see csa_index_topk)."""
+    return csa_index_topk(*args, q_group=q_group, **kw)
 
 
 def csa_index_score(q_fp4, q_scale, w, q_pos, q_seq, k_fp4, k_scale, n_entries, *, m: int,
@@ -290,8 +316,10 @@ def hca_attn_workspace(Nq: int, H: int, D: int, E_max: int, W: int) -> int:
 
 
 def csa_sparse_attn(q, q_pos, q_seq, entries, idx, cnt, window, window_base, *, W: int, scale: float | None = None,
-                    out=None, want_lse: bool = False, workspace: torch.Tensor | None = None):
-    """MQA over selected entries + window.  q [Nq,H,D] bf16; entries [B,E_max,D]; window [B,Tw,D]."""
+                    out=None, want_lse: bool = False, workspace: torch.Tensor | None = None, prep: dict | None = None):
+    """MQA over selected entries + window.  q [Nq,H,D] bf16; entries [B,E_max,D]; window [B,Tw,D].
+    prep = dict(norm, eps, rope_dims, theta): q is raw and the kernel applies csa_norm_rope's
+    transform as it loads it (csa_sparse_attn_ex)."""
     Nq, H, D = q.shape
     B, E_max, _ = entries.shape
     Tw = window.shape[1]
@@ -305,16 +333,17 @@ def csa_sparse_attn(q, q_pos, q_seq, entries, idx, cnt, window, window_base, *, 
     need = csa_sparse_attn_workspace(Nq, H, D, k, W)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    st = lib().csa_sparse_attn(Nq, H, D, k, W, scale, _ptr(q), _ptr(q_pos), _ptr(q_seq), B, E_max, _ptr(entries),
-                               _ptr(idx), _ptr(cnt), Tw, _ptr(window), _ptr(window_base), _ptr(out), _ptr(lse),
-                               _ptr(workspace), workspace.numel(), _stream(q))
+    st = lib().csa_sparse_attn_ex(_q_prep(prep), Nq, H, D, k, W, scale, _ptr(q), _ptr(q_pos), _ptr(q_seq), B, E_max,
+                                  _ptr(entries), _ptr(idx), _ptr(cnt), Tw, _ptr(window), _ptr(window_base), _ptr(out),
+                                  _ptr(lse), _ptr(workspace), workspace.numel(), _stream(q))
     _check("csa_sparse_attn", st)
     return out, lse
 
 
 def hca_attn(q, q_pos, q_seq, entries, n_entries, window, window_base, *, mprime: int, W: int,
-             scale: float | None = None, out=None, want_lse: bool = False, workspace: torch.Tensor | None = None):
-    """Dense MQA over every visible HCA entry + window."""
+             scale: float | None = None, out=None, want_lse: bool = False, workspace: torch.Tensor | None = None,
+             prep: dict | None = None):
+    """Dense MQA over every visible HCA entry + window (prep: as csa_sparse_attn)."""
     Nq, H, D = q.shape
     B, E_max, _ = entries.shape
     Tw = window.shape[1]
@@ -325,11 +354,21 @@ def hca_attn(q, q_pos, q_seq, entries, n_entries, window, window_base, *, mprime
     need = hca_attn_workspace(Nq, H, D, E_max, W)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    st = lib().hca_attn(Nq, H, D, mprime, W, scale, _ptr(q), _ptr(q_pos), _ptr(q_seq), B, E_max, _ptr(entries),
-                        _ptr(n_entries), Tw, _ptr(window), _ptr(window_base), _ptr(out), _ptr(lse),
-                        _ptr(workspace), workspace.numel(), _stream(q))
+    st = lib().hca_attn_ex(_q_prep(prep), Nq, H, D, mprime, W, scale, _ptr(q), _ptr(q_pos), _ptr(q_seq), B, E_max,
+                           _ptr(entries), _ptr(n_entries), Tw, _ptr(window), _ptr(window_base), _ptr(out), _ptr(lse),
+                           _ptr(workspace), workspace.numel(), _stream(q))
     _check("hca_attn", st)
     return out, lse
+
+
+def csa_sparse_attn_ex(prep: dict | None, *args, **kw):
+    """csa_sparse_attn with the query prepared in the kernel (prep: see csa_sparse_attn)."""
+    return csa_sparse_attn(*args, prep=prep, **kw)
+
+
+def hca_attn_ex(prep: dict | None, *args, **kw):
+    """hca_attn with the query prepared in the kernel (prep: see csa_sparse_attn)."""
+    return hca_attn(*args, prep=prep, **kw)
 
 
 def csa_grouped_out_proj(o, A, Bm, *, z=None, y=None):

@@ -222,7 +222,18 @@ csa_status csa_index_topk(int Nq, int Hi, int Di, int k, int m, const uint8_t* q
                           const float* w, const int32_t* q_pos, const int32_t* q_seq, int B, int E_max,
                           const uint8_t* k_fp4, const uint8_t* k_scale, const int32_t* n_entries, int32_t* idx_out,
                           int32_t* cnt_out, float* score_out, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  return csa_index_topk_grouped(1, Nq, Hi, Di, k, m, q_fp4, q_scale, w, q_pos, q_seq, B, E_max, k_fp4, k_scale,
+                                n_entries, idx_out, cnt_out, score_out, workspace, ws_bytes, stream);
+}
+
+csa_status csa_index_topk_grouped(int q_group, int Nq, int Hi, int Di, int k, int m, const uint8_t* q_fp4,
+                                  const uint8_t* q_scale, const float* w, const int32_t* q_pos, const int32_t* q_seq,
+                                  int B, int E_max, const uint8_t* k_fp4, const uint8_t* k_scale,
+                                  const int32_t* n_entries, int32_t* idx_out, int32_t* cnt_out, float* score_out,
+                                  void* workspace, size_t ws_bytes, cudaStream_t stream) {
   if (Nq < 0 || k < 1 || m < 1 || B < 1 || E_max < 1) return CSA_ERR_INVALID_ARG;
+  if (q_group != 1 && q_group != 2) return CSA_ERR_UNSUPPORTED;
+  if (q_group == 2 && (Hi != 64 || Di != 128)) return CSA_ERR_UNSUPPORTED;
   if (Hi < 1 || Hi > 64 || (Di != 64 && Di != 128)) return CSA_ERR_UNSUPPORTED;
   if (E_max % 8 != 0) return CSA_ERR_UNSUPPORTED;
   if (Nq == 0) return CSA_OK;
@@ -252,6 +263,7 @@ csa_status csa_index_topk(int Nq, int Hi, int Di, int k, int m, const uint8_t* q
   a.score_out = score_out;
   a.scores_ws = static_cast<float*>(workspace);
   a.E_stride = (E_max + 3) & ~3;
+  a.q_group = q_group;
   return from_cuda(launch_index_topk(a, stream));
 }
 
@@ -364,10 +376,33 @@ static csa_status attn_common(AttnArgs& a, int max_keys, cudaStream_t stream) {
   return from_cuda(launch_attention(a, max_keys, stream));
 }
 
+// The query preparation of the _ex calls (NULL: none).
+static csa_status set_q_prep(AttnArgs& a, const csa_q_prep* prep) {
+  if (prep == nullptr) return CSA_OK;
+  if (prep->rope_dims < 0 || prep->rope_dims > 64 || (prep->rope_dims & 1)) return CSA_ERR_UNSUPPORTED;
+  if (prep->norm && !(prep->eps >= 0.f)) return CSA_ERR_INVALID_ARG;
+  if (prep->rope_dims > 0 && !(prep->rope_theta > 0.f)) return CSA_ERR_INVALID_ARG;
+  a.q_prep = 1;
+  a.q_norm = prep->norm ? 1 : 0;
+  a.q_eps = prep->eps;
+  a.rope_dims = prep->rope_dims;
+  a.rope_theta = prep->rope_theta;
+  return CSA_OK;
+}
+
 csa_status csa_sparse_attn(int Nq, int H, int D, int k, int W, float scale, const void* q, const int32_t* q_pos,
                            const int32_t* q_seq, int B, int E_max, const void* entries, const int32_t* idx,
                            const int32_t* cnt, int Tw, const void* window_kv, const int32_t* window_base, void* out,
                            float* lse, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  return csa_sparse_attn_ex(nullptr, Nq, H, D, k, W, scale, q, q_pos, q_seq, B, E_max, entries, idx, cnt, Tw,
+                            window_kv, window_base, out, lse, workspace, ws_bytes, stream);
+}
+
+csa_status csa_sparse_attn_ex(const csa_q_prep* prep, int Nq, int H, int D, int k, int W, float scale, const void* q,
+                              const int32_t* q_pos, const int32_t* q_seq, int B, int E_max, const void* entries,
+                              const int32_t* idx, const int32_t* cnt, int Tw, const void* window_kv,
+                              const int32_t* window_base, void* out, float* lse, void* workspace, size_t ws_bytes,
+                              cudaStream_t stream) {
   if (k < 0) return CSA_ERR_INVALID_ARG;
   if (Nq > 0 && k > 0 && (idx == nullptr || cnt == nullptr)) return CSA_ERR_INVALID_ARG;
   AttnArgs a{};
@@ -393,6 +428,8 @@ csa_status csa_sparse_attn(int Nq, int H, int D, int k, int W, float scale, cons
   a.lse = lse;
   a.ws = workspace;
   a.ws_bytes = ws_bytes;
+  const csa_status ps = set_q_prep(a, prep);
+  if (ps != CSA_OK) return ps;
   const int max_keys = k + (W < Tw ? W : Tw);
   return attn_common(a, max_keys, stream);
 }
@@ -401,6 +438,14 @@ csa_status hca_attn(int Nq, int H, int D, int mprime, int W, float scale, const 
                     const int32_t* q_seq, int B, int E_max, const void* entries, const int32_t* n_entries, int Tw,
                     const void* window_kv, const int32_t* window_base, void* out, float* lse, void* workspace,
                     size_t ws_bytes, cudaStream_t stream) {
+  return hca_attn_ex(nullptr, Nq, H, D, mprime, W, scale, q, q_pos, q_seq, B, E_max, entries, n_entries, Tw, window_kv,
+                     window_base, out, lse, workspace, ws_bytes, stream);
+}
+
+csa_status hca_attn_ex(const csa_q_prep* prep, int Nq, int H, int D, int mprime, int W, float scale, const void* q,
+                       const int32_t* q_pos, const int32_t* q_seq, int B, int E_max, const void* entries,
+                       const int32_t* n_entries, int Tw, const void* window_kv, const int32_t* window_base, void* out,
+                       float* lse, void* workspace, size_t ws_bytes, cudaStream_t stream) {
   if (mprime < 1 || (Nq > 0 && n_entries == nullptr)) return CSA_ERR_INVALID_ARG;
   AttnArgs a{};
   a.Nq = Nq;
@@ -427,6 +472,8 @@ csa_status hca_attn(int Nq, int H, int D, int mprime, int W, float scale, const 
   a.lse = lse;
   a.ws = workspace;
   a.ws_bytes = ws_bytes;
+  const csa_status ps = set_q_prep(a, prep);
+  if (ps != CSA_OK) return ps;
   const int max_keys = E_max + (W < Tw ? W : Tw);
   return attn_common(a, max_keys, stream);
 }

@@ -27,6 +27,9 @@
 //
 // Roles (416 threads): warps 0-7 softmax + epilogue, warps 8-11 gather producers
 // (cp.async, 16-byte chunks; Q arrives by TMA), warp 12 TMEM owner and MMA issuer.
+// With one CTA per query the window starts on a tile boundary (when that adds no tile),
+// so a full tile of HCA entries or of window rows is one contiguous run of 128 rows: its
+// slabs arrive as 2-D TMA boxes instead of row gathers.
 // When a query's keys are split over several CTAs (few queries), the splits of a
 // query form a thread-block cluster: each CTA writes an
 // unnormalised fp32 partial and its (max, sum) to the workspace, the cluster
@@ -41,6 +44,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "rowprep.cuh"
 #include "tmap.h"
 
 namespace csa {
@@ -80,7 +84,11 @@ constexpr size_t kOffQ = 0;                                       // 64 KB: [8 d
 constexpr size_t kOffRing = 64 * 1024;                            // kRing x 16 KB
 constexpr size_t kOffP = kOffRing + kRing * kSlabBytes;           // kPBufs x 16 KB: [128 keys][128 B]
 constexpr size_t kOffSmall = kOffP + kPBufs * 16384;              // reductions, stats, barriers
-constexpr size_t kOffIdx = kOffSmall + 4096;                      // this CTA's slice of the index list
+// reductions and stats (832 floats), rope table (32 float2), row flags, 40 barriers, TMEM
+// slot and abort flag, laid out by AttnSmem below
+constexpr size_t kSmallUsed = 832 * 4 + 32 * 8 + 128 * kPBufs + (1 + 2 * kSlotBars + kPBufs + 2 + 2 + 1 + kPBufs + 2) * 8 + 8;
+constexpr size_t kOffIdx = kOffSmall + 5120;                      // this CTA's slice of the index list
+static_assert(kSmallUsed <= 5120, "small shared-memory region");
 constexpr int kIdxCap = 2048;
 constexpr size_t kAttnSmem = kOffIdx + 4 * kIdxCap + 1024;        // + alignment slack
 static_assert(kAttnSmem <= 227 * 1024, "shared memory budget");
@@ -104,12 +112,21 @@ struct AttnParams {
   float2* part_ml; // [Nq, splits, H]
   int rows_per_split, splits;
   int two_pass;    // every CTA's share is at most kMaxTiles2 tiles: attend_2pass
+  int align;       // tile-aligned key list: the window starts on a tile boundary
+  int tma_e;       // dense mode, entries tensor map valid: full entry tiles load by TMA
+  int tma_w;       // window tensor map valid: full window tiles load by TMA
+  int q_prep;      // q is raw: RMSNorm (q_norm) and partial RoPE are applied as it is loaded
+  int q_norm, rope_dims;
+  float q_eps, rope_theta;
   int32_t* err;
 };
 
-// A query's key list: n_sel entries, then n_win window rows.
+// A query's key list: n_sel entries (rows [0, n_sel)), then n_win window rows (rows
+// [win0, win0 + n_win)).  On the tile-aligned layout win0 is n_sel rounded up to a whole
+// tile when that costs no extra tile, so that every tile holds rows of one contiguous run;
+// rows [n_sel, win0) have no source.
 struct KeyList {
-  int b, n_sel, n_win;
+  int b, n_sel, n_win, win0;
   int64_t u_lo, wbase;
 };
 
@@ -158,7 +175,36 @@ __device__ __forceinline__ KeyList key_list(const AttnParams& p, int n, const Ke
   if (hi > kl.wbase + p.Tw - 1) hi = kl.wbase + p.Tw - 1;
   kl.u_lo = lo;
   kl.n_win = (p.W > 0 && hi >= lo) ? static_cast<int>(hi - lo + 1) : 0;
+  kl.win0 = kl.n_sel;
+  if (p.align) {
+    const int padded = (kl.n_sel + kBN - 1) / kBN * kBN;
+    const int tiles_a = padded / kBN + (kl.n_win + kBN - 1) / kBN;
+    const int tiles_u = (kl.n_sel + kl.n_win + kBN - 1) / kBN;
+    if (tiles_a <= tiles_u) kl.win0 = padded;
+  }
   return kl;
+}
+
+// A tile (rows [ts, ts + kBN) of the key list) whose rows are all present and form one
+// contiguous run of a tensor -- every row a dense-mode entry, or every row a window row --
+// loads slab by slab as 2-D TMA boxes of 128 rows x 128 bytes.  Returns the tensor map
+// and the first row's coordinate in it, or no map (the rows are gathered).  Ragged tiles
+// are always gathered: their missing rows must read as zeros, which a box cannot promise.
+struct TileBox {
+  const CUtensorMap* map;
+  int row;
+};
+
+__device__ __forceinline__ TileBox tile_box(const AttnParams& p, const KeyList& kl, const CUtensorMap& tm_e,
+                                            const CUtensorMap& tm_w, int ts, int row_end) {
+  TileBox tb{nullptr, 0};
+  if (!p.align || ts + kBN > row_end) return tb;
+  if (ts + kBN <= kl.n_sel) {
+    if (p.tma_e) tb = TileBox{&tm_e, kl.b * p.E_max + ts};
+  } else if (ts >= kl.win0) {
+    if (p.tma_w) tb = TileBox{&tm_w, kl.b * p.Tw + static_cast<int>(kl.u_lo + (ts - kl.win0) - kl.wbase)};
+  }
+  return tb;
 }
 
 __device__ __forceinline__ uint32_t sw128(int row, int chunk) {  // byte offset inside an 8-row x 128 B atom column
@@ -227,6 +273,8 @@ struct AttnSmem {
   float* l_run;      // [64]
   float* alpha;      // [64]
   float* inv_l;      // [64]
+  float* hscale;     // [64]: logit scale per head (log2 units; with the query's norm folded in)
+  float2* cs_tab;    // [32]: (cos, sin) of the query's rope pairs (query preparation)
   uint8_t* row_ok;   // [kPBufs][128]: key row has a valid source
   uint64_t* q_full;     // TMA: Q landed
   uint64_t* full;       // [kSlotBars] producers: slab landed
@@ -237,6 +285,7 @@ struct AttnSmem {
   uint64_t* o_done;     // MMA commit: PV of a tile complete
   uint64_t* row_ready;  // [kPBufs] producers: row_ok of a tile written
   uint64_t* fin;        // MMA commit: every MMA of the CTA complete
+  uint64_t* q_ready;    // softmax warps: the query prepared in place (query preparation only)
   uint32_t* tmem_slot;
   volatile int* abort_flag;
   int32_t* sidx;        // this CTA's slice of the index list
@@ -250,7 +299,9 @@ struct AttnSmem {
     l_run = m_run + 64;
     alpha = l_run + 64;
     inv_l = alpha + 64;
-    row_ok = reinterpret_cast<uint8_t*>(inv_l + 64);
+    hscale = inv_l + 64;
+    cs_tab = reinterpret_cast<float2*>(hscale + 64);
+    row_ok = reinterpret_cast<uint8_t*>(cs_tab + 32);
     uint64_t* bars = reinterpret_cast<uint64_t*>(row_ok + 128 * kPBufs);
     q_full = bars;
     full = q_full + 1;
@@ -261,17 +312,98 @@ struct AttnSmem {
     o_done = p_full + 2;
     row_ready = o_done + 1;
     fin = row_ready + kPBufs;
-    tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+    q_ready = fin + 1;
+    tmem_slot = reinterpret_cast<uint32_t*>(q_ready + 1);
     abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);
   }
 };
 
+// The query prepared in the kernel, off the MMA's critical path.  The raw query lands in
+// sQ by TMA as usual and QK starts on it at once; the preparation only has to finish the
+// part that differs:
+//   * RoPE rotates the last rope_dims channels (all in Q's last 64-dim atom, rope_dims <=
+//     64) in place; the MMA waits for them (q_ready) only before the first QK of that atom;
+//   * RMSNorm scales head row h by inv_h, which scales S^T's column h by inv_h: the softmax
+//     folds it into the logit scale (hscale[h] = scale log2(e) inv_h), computed while QK
+//     runs, instead of Q being rescaled.
+// Mathematically the query csa_norm_rope would write (a rotation commutes with a scale);
+// the rounding differs: the rotated channels are rounded to bf16 unscaled and the scale
+// is applied in float32.  The 256 softmax threads split the work as (head h = t / 4,
+// quarter c = t % 4): in the last atom, chunks 2c and 2c + 1 of row h (16 channels); for
+// the norm, 112 channels of atoms 0..6 plus those 16.  cs_tab holds the (cos, sin) of the
+// query's rope pairs; ssq the per-thread sums of squares of the raw last-atom channels.
+__device__ __forceinline__ void prep_query(const AttnParams& p, int n, uint8_t* sQ, uint64_t* q_full,
+                                           uint64_t* q_ready, float* hscale, float2* cs_tab,
+                                           volatile int* abort_flag, int warp, int lane) {
+  const int t = static_cast<int>(threadIdx.x);  // 0..255 (softmax warps)
+  const int h = t >> 2, c = t & 3;
+  const int npairs = p.rope_dims >> 1;
+  const int rope_base = kD - p.rope_dims;  // >= 448: inside the last atom
+  if (warp == 0 && lane < npairs)  // overlaps the query's load
+    cs_tab[lane] = rowprep::rope_cs(static_cast<double>(p.q_pos[n]), rowprep::inv_freq(p.rope_theta, lane, p.rope_dims));
+  const bool got = warp_wait(q_full, 0, p.err, abort_flag);
+  named_bar_sync(1, 256);  // cs_tab written
+  float ss = 0.f;
+  if (got) {
+    // last atom: 16 raw channels [448 + 16 c, 448 + 16 c + 16) of row h, rotated in place
+    uint8_t* a7 = sQ + 7 * 8192;
+    uint4* p0 = reinterpret_cast<uint4*>(a7 + sw128(h, 2 * c));
+    uint4* p1 = reinterpret_cast<uint4*>(a7 + sw128(h, 2 * c + 1));
+    const uint4 r0 = *p0, r1 = *p1;
+    const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) ss = fmaf(v[e], v[e], ss);
+    if (npairs > 0 && 448 + 16 * c + 16 > rope_base) {
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {
+        const int d = 448 + 16 * c + e;
+        if (d >= rope_base) {
+          const float2 cs = cs_tab[(d - rope_base) >> 1];
+          const float x0 = v[e], x1 = v[e + 1];
+          v[e] = fmaf(x0, cs.x, -(x1 * cs.y));
+          v[e + 1] = fmaf(x0, cs.y, x1 * cs.x);
+        }
+      }
+      *p0 = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                       pack_bf16x2(v[6], v[7]));
+      *p1 = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                       pack_bf16x2(v[14], v[15]));
+      fence_proxy_async_smem();
+    }
+  }
+  mbar_arrive(q_ready);
+  if (got) {
+    // the norm: 112 raw channels of atoms 0..6 (chunks 14 c .. 14 c + 13 of row h) while QK runs
+#pragma unroll 7
+    for (int k = 0; k < 14; ++k) {
+      const int ch = 14 * c + k;  // chunk index over atoms 0..6: atom ch / 8, chunk ch % 8
+      const uint4 r = *reinterpret_cast<const uint4*>(sQ + (ch >> 3) * 8192 + sw128(h, ch & 7));
+      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+        ss = fmaf(lo, lo, ss);
+        ss = fmaf(hi, hi, ss);
+      }
+    }
+  }
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);  // the four threads of row h are lanes 4k .. 4k + 3
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  if (c == 0) hscale[h] = p.scale_log2 * (p.q_norm ? 1.0f / sqrtf(ss / static_cast<float>(kD) + p.q_eps) : 1.f);
+}
+
 // One CTA's share of a query: rows [row_begin, row_end) of its key list, n_tiles > 0.
 // Writes the normalised output (splits == 1) or the unnormalised partial + (max, sum).
-__device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& tm_q, uint8_t* smem, uint32_t tmem,
-                                       int n, int split, const KeyList& kl, int row_begin, int row_end,
-                                       int n_tiles) {
+__device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& tm_q, const CUtensorMap& tm_e,
+                                       const CUtensorMap& tm_w, uint8_t* smem, uint32_t tmem, int n, int split,
+                                       const KeyList& kl, int row_begin, int row_end, int n_tiles) {
   const AttnSmem L(smem);
   uint8_t* sQ = L.sQ;
   uint8_t* sRing = L.sRing;
@@ -333,7 +465,8 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
         if (flag) atomicExch(p.err, CSA_DEVERR_INDEX);
         return nullptr;
       }
-      const int64_t u = kl.u_lo + (g - kl.n_sel);
+      if (g < kl.win0) return nullptr;
+      const int64_t u = kl.u_lo + (g - kl.win0);
       return p.window + (static_cast<size_t>(kl.b) * p.Tw + static_cast<size_t>(u - kl.wbase)) * kD;
     };
     bool ok = true;
@@ -346,6 +479,7 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
       const bool valid = src_row != nullptr;
       const uint16_t* src = valid ? src_row : p.entries;
       const unsigned long long src_ll = reinterpret_cast<unsigned long long>(src);
+      const TileBox box = tile_box(p, kl, tm_e, tm_w, row_begin + tile * kBN, row_end);
       for (int ka = 0; ka < kSlabs; ++ka, ++j) {
         const int slot = j % kRing;
         if (!warp_wait(&slot_free[slot], ((j / kRing) & 1) ^ 1, p.err, abort_flag)) {
@@ -360,6 +494,15 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
           if (ptid == 0 && tile < 8) CSA_T(tslot, 8 + tile);
         }
         const uint32_t dst = smem_u32(sRing + slot * kSlabBytes);
+        if (box.map != nullptr) {  // one box per slab; every producer thread still arrives once
+          if (ptid == 0) {
+            mbar_arrive_expect_tx(&full[slot], kSlabBytes);
+            tma_load_2d(dst, box.map, &full[slot], ka * 128, box.row);
+          } else {
+            mbar_arrive(&full[slot]);
+          }
+          continue;
+        }
         for (int qb = 0; qb < 8 * nrows; qb += 32) {  // warp-uniform trip count: every lane shuffles
           const int q = qb + lane;                      // chunk q: row r0 + q / 8, 16 bytes q % 8
           const bool in = q < 8 * nrows;
@@ -384,6 +527,9 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     constexpr uint32_t idesc_pv = idesc_bf16(128, kH, true, true);
     const uint32_t q0 = smem_u32(sQ), ring0 = smem_u32(sRing), p0 = smem_u32(sP);
     bool ok = warp_wait(q_full, 0, p.err, abort_flag);
+    // query preparation: the rotated atoms are ready for the MMA once q_ready completes
+    const int rope_atom = p.q_prep && p.rope_dims > 0 ? (kD - p.rope_dims) / 64 : kSlabs;
+    bool q_ready_seen = rope_atom >= kSlabs;
     int j = 0;
     for (int st = 0; ok && st < 2 * n_tiles; ++st) {
       int tile;
@@ -398,6 +544,13 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
           if (!warp_wait(&full[slot], (j / kRing) & 1, p.err, abort_flag)) {
             ok = false;
             break;
+          }
+          if (!q_ready_seen && ka >= rope_atom) {  // the query's rotated channels are written
+            q_ready_seen = true;
+            if (!warp_wait(L.q_ready, 0, p.err, abort_flag)) {
+              ok = false;
+              break;
+            }
           }
           if (lane == 0 && tslot == 4 && j < 64) CSA_T(12, j);
           fence_proxy_async_smem();  // the producers' cp.async writes, seen through the barrier
@@ -459,6 +612,12 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     // ------------------------------------------------------------ softmax (warps 0-7)
     // thread = one key row of the tile (TMEM lane 32*(warp%4)+lane) and 32 heads
     // (hh = warp/4 selects heads 0-31 or 32-63).
+    if (p.q_prep)
+      prep_query(p, n, sQ, q_full, L.q_ready, L.hscale, L.cs_tab, abort_flag, warp, lane);
+    else if (threadIdx.x < kH)
+      L.hscale[threadIdx.x] = p.scale_log2;
+    named_bar_sync(1, 256);
+    const float* hscale = L.hscale;
     const int q4 = warp & 3, hh = warp >> 2;
     const int t = 32 * q4 + lane;
     const int h0 = 32 * hh;
@@ -492,7 +651,13 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
         tmem_ld16(s_addr + 16, sr + 16);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = valid ? __uint_as_float(sr[i]) * p.scale_log2 : -INFINITY;
+        for (int i = 0; i < 32; i += 4) {
+          const float4 hs = *reinterpret_cast<const float4*>(hscale + h0 + i);
+          x[i] = valid ? __uint_as_float(sr[i]) * hs.x : -INFINITY;
+          x[i + 1] = valid ? __uint_as_float(sr[i + 1]) * hs.y : -INFINITY;
+          x[i + 2] = valid ? __uint_as_float(sr[i + 2]) * hs.z : -INFINITY;
+          x[i + 3] = valid ? __uint_as_float(sr[i + 3]) * hs.w : -INFINITY;
+        }
       }
       bool over = false;
 #pragma unroll
@@ -524,7 +689,13 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
         tmem_ld16(s_addr + 16, sr + 16);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = valid ? __uint_as_float(sr[i]) * p.scale_log2 : -INFINITY;
+        for (int i = 0; i < 32; i += 4) {
+          const float4 hs = *reinterpret_cast<const float4*>(hscale + h0 + i);
+          x[i] = valid ? __uint_as_float(sr[i]) * hs.x : -INFINITY;
+          x[i + 1] = valid ? __uint_as_float(sr[i + 1]) * hs.y : -INFINITY;
+          x[i + 2] = valid ? __uint_as_float(sr[i + 2]) * hs.z : -INFINITY;
+          x[i + 3] = valid ? __uint_as_float(sr[i + 3]) * hs.w : -INFINITY;
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -678,9 +849,10 @@ __device__ __forceinline__ Slot2 slot_v2(int v, int nK) {
 // L2, into the ring slots the K pass frees, while the softmax works, and PV accumulates
 // O^T in columns [256, 512).  Same outputs as attend(): the normalised result or the
 // unnormalised partial with its (max, sum).
-__device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensorMap& tm_q, uint8_t* smem,
-                                             uint32_t tmem, int n, int split, const KeyList& kl, int row_begin,
-                                             int row_end, int n_tiles) {
+__device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensorMap& tm_q, const CUtensorMap& tm_e,
+                                             const CUtensorMap& tm_w, uint8_t* smem, uint32_t tmem, int n,
+                                             int split, const KeyList& kl, int row_begin, int row_end,
+                                             int n_tiles) {
   const AttnSmem L(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tslot = blockIdx.x < 2 ? 4 + static_cast<int>(blockIdx.x) : -1;
@@ -712,7 +884,8 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
         if (flag) atomicExch(p.err, CSA_DEVERR_INDEX);
         return nullptr;
       }
-      const int64_t u = kl.u_lo + (g - kl.n_sel);
+      if (g < kl.win0) return nullptr;
+      const int64_t u = kl.u_lo + (g - kl.win0);
       return p.window + (static_cast<size_t>(kl.b) * p.Tw + static_cast<size_t>(u - kl.wbase)) * kD;
     };
     bool ok = true;
@@ -724,6 +897,7 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
       const uint16_t* src_row = row_src(tile, !is_v);
       const bool valid = src_row != nullptr;
       const unsigned long long src_ll = reinterpret_cast<unsigned long long>(valid ? src_row : p.entries);
+      const TileBox box = tile_box(p, kl, tm_e, tm_w, row_begin + tile * kBN, row_end);
       if (ptid == 0) CSA_T(tslot, 8 + st);
       if (!is_v && lane < nrows) {  // published before this tile's first slab is issued
         L.row_ok[tile * 128 + r0 + lane] = valid ? 1 : 0;
@@ -745,6 +919,15 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
         }
         if (ptid == 0 && tslot == 4 && j < 64) CSA_T(10, j);
         const uint32_t dst = smem_u32(smem + sl.off);
+        if (box.map != nullptr) {
+          if (ptid == 0) {
+            mbar_arrive_expect_tx(&L.full[sl.bar], kSlabBytes);
+            tma_load_2d(dst, box.map, &L.full[sl.bar], ka * 128, box.row);
+          } else {
+            mbar_arrive(&L.full[sl.bar]);
+          }
+          continue;
+        }
         for (int qb = 0; qb < 8 * nrows; qb += 32) {
           const int q = qb + lane;
           const bool in = q < 8 * nrows;
@@ -768,6 +951,8 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
     const uint32_t base = smem_u32(smem), q0 = smem_u32(L.sQ), p0 = smem_u32(L.sP);
     const int nK = kSlabs * n_tiles;
     bool ok = warp_wait(L.q_full, 0, p.err, L.abort_flag);
+    const int rope_atom = p.q_prep && p.rope_dims > 0 ? (kD - p.rope_dims) / 64 : kSlabs;
+    bool q_ready_seen = rope_atom >= kSlabs;
     if (lane == 0) CSA_T(tslot, 1);
     for (int tile = 0; ok && tile < n_tiles; ++tile) {  // K pass: S^T[tile] = K Q^T
       for (int ka = 0; ka < kSlabs; ++ka) {
@@ -776,6 +961,13 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
         if (!warp_wait(&L.full[sl.bar], sl.parity, p.err, L.abort_flag)) {
           ok = false;
           break;
+        }
+        if (!q_ready_seen && ka >= rope_atom) {  // the query's rotated channels are written
+          q_ready_seen = true;
+          if (!warp_wait(L.q_ready, 0, p.err, L.abort_flag)) {
+            ok = false;
+            break;
+          }
         }
         if (lane == 0 && tslot == 4 && j < 64) CSA_T(12, j);
         fence_proxy_async_smem();
@@ -833,6 +1025,12 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
   } else {
     // ------------------------------------------------------------ softmax (warps 0-7)
     // thread = key row t of each tile (TMEM lane 32 (warp % 4) + lane) and 32 heads
+    if (p.q_prep)
+      prep_query(p, n, L.sQ, L.q_full, L.q_ready, L.hscale, L.cs_tab, L.abort_flag, warp, lane);
+    else if (threadIdx.x < kH)
+      L.hscale[threadIdx.x] = p.scale_log2;
+    named_bar_sync(1, 256);
+    const float* hscale = L.hscale;
     const int q4 = warp & 3, hh = warp >> 2;
     const int t = 32 * q4 + lane;
     const int h0 = 32 * hh;
@@ -859,7 +1057,13 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
       tmem_wait_ld();
       if (valid) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx[i] = fmaxf(mx[i], __uint_as_float(sr[i]) * p.scale_log2);
+        for (int i = 0; i < 32; i += 4) {
+          const float4 hs = *reinterpret_cast<const float4*>(hscale + h0 + i);
+          mx[i] = fmaxf(mx[i], __uint_as_float(sr[i]) * hs.x);
+          mx[i + 1] = fmaxf(mx[i + 1], __uint_as_float(sr[i + 1]) * hs.y);
+          mx[i + 2] = fmaxf(mx[i + 2], __uint_as_float(sr[i + 2]) * hs.z);
+          mx[i + 3] = fmaxf(mx[i + 3], __uint_as_float(sr[i + 3]) * hs.w);
+        }
       }
     }
     if (ok) {
@@ -888,10 +1092,11 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           const float4 mm = *reinterpret_cast<const float4*>(L.m_run + h0 + i);
-          x[i] = fast_exp2(fmaf(__uint_as_float(sr[i]), p.scale_log2, -mm.x));
-          x[i + 1] = fast_exp2(fmaf(__uint_as_float(sr[i + 1]), p.scale_log2, -mm.y));
-          x[i + 2] = fast_exp2(fmaf(__uint_as_float(sr[i + 2]), p.scale_log2, -mm.z));
-          x[i + 3] = fast_exp2(fmaf(__uint_as_float(sr[i + 3]), p.scale_log2, -mm.w));
+          const float4 hs = *reinterpret_cast<const float4*>(hscale + h0 + i);
+          x[i] = fast_exp2(fmaf(__uint_as_float(sr[i]), hs.x, -mm.x));
+          x[i + 1] = fast_exp2(fmaf(__uint_as_float(sr[i + 1]), hs.y, -mm.y));
+          x[i + 2] = fast_exp2(fmaf(__uint_as_float(sr[i + 2]), hs.z, -mm.z));
+          x[i + 3] = fast_exp2(fmaf(__uint_as_float(sr[i + 3]), hs.w, -mm.w));
         }
       } else {
 #pragma unroll
@@ -996,6 +1201,7 @@ __device__ __forceinline__ uint32_t attn_setup(uint8_t* smem) {
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(L.q_ready, 256);
     for (int i = 0; i < kSlotBars; ++i) {
       mbar_init(&full[i], kProdThreads);
       mbar_init(&slot_free[i], 1);
@@ -1091,11 +1297,17 @@ __device__ __forceinline__ void merge_partials(const AttnParams& p, int n, int h
   }
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_constant__ CUtensorMap tm_q, AttnParams p) {
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_e,
+                const __grid_constant__ CUtensorMap tm_w, AttnParams p) {
   CSA_TB(0);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  if (threadIdx.x == 0) prefetch_tmap(&tm_q);
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tm_q);
+    if (p.tma_e) prefetch_tmap(&tm_e);
+    if (p.tma_w) prefetch_tmap(&tm_w);
+  }
   const uint32_t tmem = attn_setup(smem);
   const int n = blockIdx.x / p.splits;
   const int split = blockIdx.x % p.splits;  // the CTA's rank in its cluster when splits > 1
@@ -1108,7 +1320,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
   int row_begin = 0, row_end = 0, n_tiles = 0;
   if (seq_ok) {
     kl = key_list(p, n, meta);
-    const int nk = kl.n_sel + kl.n_win;
+    const int nk = kl.win0 + kl.n_win;
     row_begin = split * p.rows_per_split;
     row_end = min(nk, row_begin + p.rows_per_split);
     n_tiles = row_end > row_begin ? (row_end - row_begin + kBN - 1) / kBN : 0;
@@ -1116,9 +1328,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
 
   if (n_tiles > 0) {
     if (p.two_pass)
-      attend_2pass(p, tm_q, smem, tmem, n, split, kl, row_begin, row_end, n_tiles);
+      attend_2pass(p, tm_q, tm_e, tm_w, smem, tmem, n, split, kl, row_begin, row_end, n_tiles);
     else
-      attend(p, tm_q, smem, tmem, n, split, kl, row_begin, row_end, n_tiles);
+      attend(p, tm_q, tm_e, tm_w, smem, tmem, n, split, kl, row_begin, row_end, n_tiles);
   }
   tc_fence_before();
   __syncthreads();
@@ -1219,15 +1431,44 @@ cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s) {
   p.window_base = a.window_base;
   p.out = a.out;
   p.lse = a.lse;
+  p.q_prep = a.q_prep;
+  p.q_norm = a.q_norm;
+  p.q_eps = a.q_eps;
+  p.rope_dims = a.rope_dims;
+  p.rope_theta = a.rope_theta;
   p.err = device_error_word();
   const int splits = split_count(a.Nq, max_keys);
   p.splits = splits;
-  p.rows_per_split = std::max(32, (((max_keys + splits - 1) / splits) + 31) / 32 * 32);
+  // One CTA per query: the tile-aligned layout, when it adds no tile at the largest key
+  // list; full tiles of contiguous rows then load by TMA.  (Not in batch-invariant mode,
+  // where a query's tiles, and so its rounding, must not depend on the call's sizes.)
+  const int max_sel = std::min(a.dense ? a.E_max : a.k, max_keys);
+  const int max_win = max_keys - max_sel;
+  const int pad_keys = (max_sel + kBN - 1) / kBN * kBN + max_win;
+  p.align = (splits == 1 && !batch_invariant() && (pad_keys + kBN - 1) / kBN <= (max_keys + kBN - 1) / kBN) ? 1 : 0;
+  const int rows = p.align ? pad_keys : max_keys;
+  p.rows_per_split = std::max(32, (((rows + splits - 1) / splits) + 31) / 32 * 32);
   p.two_pass = p.rows_per_split <= kMaxTiles2 * kBN ? 1 : 0;
   if (static_cast<int64_t>(a.Nq) * kH >= INT32_MAX) return cudaErrorInvalidValue;  // 32-bit TMA row coordinate
   CUtensorMap tm_q;  // the queries as 64-row x 128-byte boxes
   if (!encode_2d_u8(&tm_q, a.q, kD * 2, static_cast<uint64_t>(a.Nq) * kH, 128, kH, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  // entry and window rows as 128-row x 128-byte boxes (one slab of a tile); a map that
+  // cannot be encoded (unaligned base, too many rows for a 32-bit coordinate) leaves its
+  // tiles on the gather path
+  CUtensorMap tm_e{}, tm_w{};
+  const auto aligned16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
+  const int64_t e_rows = static_cast<int64_t>(a.B) * a.E_max, w_rows = static_cast<int64_t>(a.B) * a.Tw;
+  p.tma_e = (p.align && a.dense && e_rows > 0 && e_rows < INT32_MAX && aligned16(a.entries) &&
+             encode_2d_u8(&tm_e, a.entries, kD * 2, static_cast<uint64_t>(e_rows), 128, kBN,
+                          CU_TENSOR_MAP_SWIZZLE_128B))
+                ? 1
+                : 0;
+  p.tma_w = (p.align && a.window != nullptr && w_rows > 0 && w_rows < INT32_MAX && aligned16(a.window) &&
+             encode_2d_u8(&tm_w, a.window, kD * 2, static_cast<uint64_t>(w_rows), 128, kBN,
+                          CU_TENSOR_MAP_SWIZZLE_128B))
+                ? 1
+                : 0;
   if (splits > 1) {
     const size_t o_bytes = static_cast<size_t>(a.Nq) * splits * kH * kD * sizeof(float);
     uintptr_t base = reinterpret_cast<uintptr_t>(a.ws);
@@ -1238,7 +1479,7 @@ cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s) {
   cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(attn_kernel), kAttnSmem, g_attn_smem);
   if (e != cudaSuccess) return e;
   return launch_pdl_cluster(attn_kernel, dim3(a.Nq * splits), dim3(kAttnThreads), kAttnSmem,
-                            static_cast<unsigned>(splits), s, tm_q, p);
+                            static_cast<unsigned>(splits), s, tm_q, tm_e, tm_w, p);
 }
 
 }  // namespace csa

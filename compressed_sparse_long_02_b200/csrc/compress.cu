@@ -32,12 +32,11 @@
 #include "internal.h"
 #include "mxfp4.cuh"
 #include "ptx.cuh"
+#include "rowprep.cuh"
 
 namespace csa {
 namespace {
 
-constexpr double kTwoPi = 6.283185307179586476925286766559;
-constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kPoolThreads = 256;  // 8 warps
 // slots loaded together before any is consumed: 4, fewer when a lane's row slice is
@@ -46,16 +45,6 @@ constexpr int kPoolThreads = 256;  // 8 warps
 template <int kWords>
 constexpr int pool_chunk() {
   return kWords >= 32 ? 1 : (kWords >= 16 ? 2 : 4);
-}
-
-// cos / sin of pos * inv_freq: the angle reduced modulo 2 pi in double, then a float sincos
-__device__ __forceinline__ float2 rope_cs(double pos, double inv_freq) {
-  const double ang = pos * inv_freq;
-  const double k = rint(ang * kInvTwoPi);
-  const float r = static_cast<float>(fma(-k, kTwoPi, ang));
-  float s, c;
-  sincosf(r, &s, &c);
-  return make_float2(c, s);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -100,51 +89,8 @@ struct RowBits {
   }
 };
 
-// 1 / sqrt(mean of squares + eps) of a row held CPT channels per lane (all 32 lanes call it)
-template <int CPT>
-__device__ __forceinline__ float row_inv_rms(const float (&v)[CPT], int C, float eps) {
-  float ss = 0.f;
-#pragma unroll
-  for (int e = 0; e < CPT; ++e) ss = fmaf(v[e], v[e], ss);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  return 1.0f / sqrtf(ss / static_cast<float>(C) + eps);
-}
-
-// Partial RoPE at position pos of the lane's channels [c0, c0 + CPT): pair (2i, 2i+1) of
-// the last rope_dims channels turns by pos * inv_freq[i].  The angles are spread over the
-// warp (lane l computes pairs l, l + 32, ...) and handed to the lanes that own the pairs
-// by shuffles, so no lane computes more than ceil(pairs / 32) of them.  All 32 lanes call.
-template <int CPT>
-__device__ __forceinline__ void rope_lane(float (&v)[CPT], int c0, int C, int rope_dims, double pos,
-                                          const double* inv_freq) {
-  const int npairs = rope_dims >> 1;
-  if (npairs == 0) return;
-  const int lane = threadIdx.x & 31;
-  const int rope_base = C - rope_dims;
-  const int first_lane = rope_base / CPT;  // lanes holding rope channels: [first_lane, 32)
-  for (int base = 0; base < npairs; base += 32) {
-    const int i = base + lane;
-    const float2 cs = i < npairs ? rope_cs(pos, inv_freq[i]) : make_float2(1.f, 0.f);
-    // pair i sits in lane first_lane + (2 i) / CPT (the rope channels start on a lane boundary
-    // when CPT divides rope_base; otherwise the lane's own index test below still holds)
-#pragma unroll
-    for (int e = 0; e < CPT; e += 2) {
-      const int c = c0 + e;
-      const int pi = (c - rope_base) >> 1;       // this lane's pair at slot e (may be out of range)
-      const int src = (pi - base) & 31;          // lane holding its angle in this round
-      const float cx = __shfl_sync(0xffffffffu, cs.x, src);
-      const float sx = __shfl_sync(0xffffffffu, cs.y, src);
-      if (c >= rope_base && pi >= base && pi < base + 32) {
-        const float r0 = fmaf(v[e], cx, -(v[e + 1] * sx));
-        const float r1 = fmaf(v[e], sx, v[e + 1] * cx);
-        v[e] = r0;
-        v[e + 1] = r1;
-      }
-    }
-  }
-  (void)first_lane;
-}
+using rowprep::rope_lane;
+using rowprep::row_inv_rms;
 
 // RMSNorm (optional) + RoPE of one row, stored as bf16 at out_row + lane's channels
 template <int CPT>
@@ -244,7 +190,7 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(PoolArgs a) {
   double* inv_freq = reinterpret_cast<double*>(pool_smem);
   float* part = reinterpret_cast<float*>(pool_smem + (a.rope_dims / 2) * sizeof(double));  // [kSplit][3][C]
   for (int i = threadIdx.x; i < a.rope_dims / 2; i += kPoolThreads)
-    inv_freq[i] = pow(static_cast<double>(a.theta), -2.0 * i / a.rope_dims);
+    inv_freq[i] = rowprep::inv_freq(a.theta, i, a.rope_dims);
   __syncthreads();
   griddep_enter();
 
@@ -388,7 +334,7 @@ __global__ void __launch_bounds__(kPoolThreads) norm_rope_kernel(NormRopeArgs a)
   extern __shared__ __align__(16) uint8_t nr_smem[];
   double* inv_freq = reinterpret_cast<double*>(nr_smem);
   for (int i = threadIdx.x; i < a.rope_dims / 2; i += blockDim.x)
-    inv_freq[i] = pow(static_cast<double>(a.theta), -2.0 * i / a.rope_dims);
+    inv_freq[i] = rowprep::inv_freq(a.theta, i, a.rope_dims);
   __syncthreads();
   griddep_enter();
   const int64_t row = blockIdx.x;

@@ -82,28 +82,45 @@ struct IndexParams {
 // warps select.
 constexpr int kFuseThreads = 256;
 constexpr int kFuseStages = 6;
-template <int kFuseC, int kFuseEPT>
+// The grouped variant (kQ = 2): the two consecutive query rows of a group belong to one
+// sequence (several new tokens of a sequence at decode) and share every key tile: one
+// N = 128 MMA per K step scores both queries' 64 heads.  Its accumulators are 128
+// columns wide, so it takes 512 TMEM columns and runs one CTA per SM (deeper key ring,
+// more tiles per CTA).
+constexpr int kQStages = 16;
+constexpr int kQMaxTiles = 64;
+template <int kFuseC, int kFuseEPT, int kQ = 1>
 struct IndexShape {
   static constexpr bool kFuse = kFuseC > 0;
   static constexpr int kThreads = kFuse ? kFuseThreads : kIdxThreads;
-  static constexpr int kSt = kFuse ? kFuseStages : kStages;
-  static constexpr int kMaxTiles = kFuse ? kFuseThreads * kFuseEPT / kTileE : kMaxTilesPerCta;
-  static constexpr int kRawSf = kFuse ? 0 : kMaxTilesPerCta;  // raw scale bytes for Di = 64 (not fused)
+  static constexpr int kSt = kFuse ? kFuseStages : (kQ > 1 ? kQStages : kStages);
+  static constexpr int kMaxTiles = kFuse ? kFuseThreads * kFuseEPT / kTileE : (kQ > 1 ? kQMaxTiles : kMaxTilesPerCta);
+  static constexpr int kRawSf = (kFuse || kQ > 1) ? 0 : kMaxTilesPerCta;  // raw scale bytes for Di = 64
   static constexpr int kSlice = kFuse ? kFuseThreads * kFuseEPT : 0;
-  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kSt) * 8192 + 4096 + static_cast<size_t>(kMaxTiles) * 512 +
-                                  static_cast<size_t>(kRawSf) * 256 + 512 + 256 + 512 + static_cast<size_t>(kSlice) * 4;
+  static constexpr uint32_t kTmem = kQ > 1 ? 512 : kTmemCols;
+  static constexpr uint32_t kAccCols = 64 * kQ;                 // one accumulator: kQ x 64 heads
+  static constexpr uint32_t kColSFA = kAccCols * kAccBufs;      // key scale-factor ring
+  static constexpr uint32_t kColSFB = kColSFA + 4 * kSfRing;    // query scale factors (4 columns)
+  static_assert(kColSFB + 4 <= kTmem, "TMEM budget");
+  static constexpr int kMinBlocks = kQ > 1 ? 1 : 2;
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kSt) * 8192 + 4096 * kQ +
+                                  static_cast<size_t>(kMaxTiles) * 512 + static_cast<size_t>(kRawSf) * 256 + 512 +
+                                  256 * kQ + 512 + static_cast<size_t>(kSlice) * 4;
 };
 
 // kHi: number of indexer heads fixed at compile time (the head chain is straight-line
 // code), or 0 to take it from p.Hi at run time.  kRawQ: the query arrives unencoded and
 // the epilogue warps encode it to MXFP4 (the same rule as quantize_mxfp4_kernel) into
-// the MMA's B operand and scale factors before the first tile.
-template <int kHi, bool kRawQ, int kFuseC = 0, int kFuseEPT = 8>
-__global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT>::kThreads, 2)
+// the MMA's B operand and scale factors before the first tile.  kQ: queries per CTA
+// sharing the key tiles (1, or 2 for the grouped variant).
+template <int kHi, bool kRawQ, int kFuseC = 0, int kFuseEPT = 8, int kQ = 1>
+__global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT, kQ>::kThreads, IndexShape<kFuseC, kFuseEPT, kQ>::kMinBlocks)
     index_score_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                        IndexParams p) {
-  using Shape = IndexShape<kFuseC, kFuseEPT>;
+  using Shape = IndexShape<kFuseC, kFuseEPT, kQ>;
   constexpr bool kFuse = Shape::kFuse;
+  static_assert(kQ == 1 || (kQ == 2 && kHi == 64 && !kRawQ && kFuseC == 0), "grouped: 64 heads, encoded queries");
+  constexpr uint32_t kColSFA = Shape::kColSFA, kColSFB = Shape::kColSFB, kAccCols = Shape::kAccCols;
   constexpr int kStages = Shape::kSt;  // shadows the plain kernel's depth in this body
   // epilogue warps: two groups of four (warps 2-9); the fused kernel one (warps 2-5)
   constexpr int kEpiGroups = kFuse ? 1 : 2;
@@ -116,12 +133,12 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT>::kThreads, 2)
 
   // shared memory carve-up
   uint8_t* sA = smem;                                    // kStages x 8 KB (1024-aligned)
-  uint8_t* sB = sA + kStages * 8192;                     // 4 KB
-  uint8_t* sSF = sB + 4096;                              // kMaxTiles x 512: key scales, scale-factor layout
+  uint8_t* sB = sA + kStages * 8192;                     // kQ x 4 KB
+  uint8_t* sSF = sB + 4096 * kQ;                         // kMaxTiles x 512: key scales, scale-factor layout
   uint8_t* sSFraw = sSF + Shape::kMaxTiles * 512;        // kRawSf x 256: raw key scales when Di = 64
   uint8_t* sSFB = sSFraw + Shape::kRawSf * 256;          // 512
-  float* sW = reinterpret_cast<float*>(sSFB + 512);      // [64] head weights
-  float* sSlice = sW + 64;                               // fused: this CTA's scores [kSlice]
+  float* sW = reinterpret_cast<float*>(sSFB + 512);      // [kQ][64] head weights
+  float* sSlice = sW + 64 * kQ;                          // fused: this CTA's scores [kSlice]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sSlice + Shape::kSlice);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
@@ -152,7 +169,7 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT>::kThreads, 2)
     prefetch_tmap(&tm_q);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(tmem_slot, Shape::kTmem);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -162,13 +179,37 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT>::kThreads, 2)
   griddep_enter();
   CSA_TB(1);
 
-  const int q = kFuse ? static_cast<int>(blockIdx.x) / kFuseC : static_cast<int>(blockIdx.x) / p.splits;
+  // the CTA's first query row (kQ > 1: the group's), and its split of the entry range
+  const int q = kQ * (kFuse ? static_cast<int>(blockIdx.x) / kFuseC : static_cast<int>(blockIdx.x) / p.splits);
   const int split = kFuse ? static_cast<int>(blockIdx.x) % kFuseC : static_cast<int>(blockIdx.x) % p.splits;
   const int seq = p.q_seq[q];
   const bool seq_ok = seq >= 0 && seq < p.B;
   if (!seq_ok && threadIdx.x == 0 && split == 0) atomicExch(p.err, CSA_DEVERR_INDEX);  // produce nothing
-  const int nvis = seq_ok ? min(visible_entries(p.q_pos[q], p.m, p.n_entries[seq]), p.E_max) : 0;
+  const int nvis0 = seq_ok ? min(visible_entries(p.q_pos[q], p.m, p.n_entries[seq]), p.E_max) : 0;
   const int tiles_per_cta = kFuse ? Shape::kMaxTiles : p.tiles_per_cta;
+  // grouped: the second query row, scored from the same key tiles when it names the same
+  // sequence; a row naming another sequence is recorded as an error and gets -inf for
+  // every entry visible to it (in this CTA's share), so that its selection is defined
+  int nvis1 = 0;
+  if constexpr (kQ > 1) {
+    const int q1 = q + 1;
+    if (q1 < p.Nq) {
+      const int seq1 = p.q_seq[q1];
+      const bool ok1 = seq1 >= 0 && seq1 < p.B;
+      const int nv1 = ok1 ? min(visible_entries(p.q_pos[q1], p.m, p.n_entries[seq1]), p.E_max) : 0;
+      if (seq_ok && seq1 == seq) {
+        nvis1 = nv1;
+      } else {
+        if (threadIdx.x == 0 && split == 0) atomicExch(p.err, CSA_DEVERR_INDEX);
+        const int e_lo = split * tiles_per_cta * kTileE, e_hi = min(nv1, e_lo + tiles_per_cta * kTileE);
+        for (int e = e_lo + static_cast<int>(threadIdx.x); e < e_hi; e += static_cast<int>(blockDim.x)) {
+          p.scores[static_cast<size_t>(q1) * p.E_stride + e] = -INFINITY;
+          if (p.score_out) p.score_out[static_cast<size_t>(q1) * p.E_max + e] = -INFINITY;
+        }
+      }
+    }
+  }
+  const int nvis = max(nvis0, nvis1);
   const int t_begin = split * tiles_per_cta;
   // fused: a query with at most k visible entries takes all of them (no scoring; the same
   // for every CTA of the cluster, so none reaches a cluster barrier below)
@@ -230,9 +271,9 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT>::kThreads, 2)
       uint32_t words[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int r = lane + 32 * i;
+        const int r = lane + 32 * i;  // B row: head r % Hi of query q + r / Hi
         uint32_t v = 0;
-        if (r < Hi) {
+        if (r < kQ * Hi && q + r / Hi < p.Nq) {
           const uint8_t* src = p.q_scale + (static_cast<size_t>(q) * Hi + r) * sf_row;
           for (int b = 0; b < sf_row; ++b) v |= static_cast<uint32_t>(src[b]) << (8 * b);
         }
@@ -265,7 +306,7 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT>::kThreads, 2)
         const uint32_t a0 = smem_u32(sA + st * 8192), b0 = smem_u32(sB);
         for (int kh = 0; kh < p.Di / 64; ++kh) {
           const uint32_t sf_id = 2 * kh;  // byte of the scale column holding blocks 2kh, 2kh+1
-          mma_mxf4(tmem + 64 * buf, smem_desc(a0 + 32 * kh, 0, sbo, swz), smem_desc(b0 + 32 * kh, 0, sbo, swz),
+          mma_mxf4(tmem + kAccCols * buf, smem_desc(a0 + 32 * kh, 0, sbo, swz), smem_desc(b0 + 32 * kh, 0, sbo, swz),
                    idesc_mxf4(kTileE, p.N, sf_id, sf_id), kh > 0 ? 1u : 0u, sfa | (sf_id << 30),
                    (tmem + kColSFB) | (sf_id << 30));
         }
@@ -278,9 +319,9 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT>::kThreads, 2)
   } else if (n_tiles > 0 && warp < 2 + kEpiWarps) {
     // ------------------------------------------------------------ epilogue (warps 2 .. 1 + kEpiWarps)
     const int ew = warp - 2;
-    if (ew * 32 + lane < 64) {
-      const int h = ew * 32 + lane;
-      sW[h] = h < Hi ? __ldg(p.w + static_cast<size_t>(q) * Hi + h) : 0.f;
+    if (ew * 32 + lane < 64 * kQ) {  // weights of head h % 64 of query q + h / 64
+      const int h = ew * 32 + lane, hq = h & 63;
+      sW[h] = (hq < Hi && q + (h >> 6) < p.Nq) ? __ldg(p.w + static_cast<size_t>(q + (h >> 6)) * Hi + hq) : 0.f;
     }
     if (kRawQ) {
       // Encode the query (Hi rows x Di) into the B operand: K-major, the 16-byte chunk c of
@@ -354,35 +395,38 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT>::kThreads, 2)
       if (!warp_wait(&acc_full[buf], (it / kAccBufs) & 1, p.err, abort_flag)) break;
       if (sub == 0 && lane == 0 && it < 16 && tslot == 0) CSA_T(6, it);
       tc_fence_after();
-      uint32_t acc[64];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + 64 * buf;
+      uint32_t acc[64 * kQ];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + kAccCols * buf;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (16 * c < Hi) tmem_ld16(taddr + 16 * c, acc + 16 * c);
+      for (int c = 0; c < 4 * kQ; ++c)
+        if (16 * (c & 3) < Hi) tmem_ld16(taddr + 16 * c, acc + 16 * c);
       tmem_wait_ld();
       if (sub == 0 && lane == 0 && it < 16 && tslot == 0) CSA_T(7, it);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
-      float s = 0.f;
-#pragma unroll
-      for (int h = 0; h < 64; h += 4) {
-        if (h < Hi) {
-          const float4 w4 = *reinterpret_cast<const float4*>(sW + h);
-          s = fmaf(w4.x, fmaxf(__uint_as_float(acc[h]), 0.f), s);
-          if (h + 1 < Hi) s = fmaf(w4.y, fmaxf(__uint_as_float(acc[h + 1]), 0.f), s);
-          if (h + 2 < Hi) s = fmaf(w4.z, fmaxf(__uint_as_float(acc[h + 2]), 0.f), s);
-          if (h + 3 < Hi) s = fmaf(w4.w, fmaxf(__uint_as_float(acc[h + 3]), 0.f), s);
-        }
-      }
       const int e = (t_begin + it) * kTileE + 32 * sub + lane;
-      if (sub == 0 && lane == 0 && it < 16) CSA_T(tslot, 48 + it);
-      if (e < nvis) {
-        if constexpr (kFuse)
-          sSlice[e - t_begin * kTileE] = s;
-        else
-          p.scores[static_cast<size_t>(q) * p.E_stride + e] = s;
-        if (p.score_out) p.score_out[static_cast<size_t>(q) * p.E_max + e] = s;
+#pragma unroll
+      for (int j = 0; j < kQ; ++j) {  // query q + j: columns [64 j, 64 j + Hi) of the accumulator
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < 64; h += 4) {
+          if (h < Hi) {
+            const float4 w4 = *reinterpret_cast<const float4*>(sW + 64 * j + h);
+            s = fmaf(w4.x, fmaxf(__uint_as_float(acc[64 * j + h]), 0.f), s);
+            if (h + 1 < Hi) s = fmaf(w4.y, fmaxf(__uint_as_float(acc[64 * j + h + 1]), 0.f), s);
+            if (h + 2 < Hi) s = fmaf(w4.z, fmaxf(__uint_as_float(acc[64 * j + h + 2]), 0.f), s);
+            if (h + 3 < Hi) s = fmaf(w4.w, fmaxf(__uint_as_float(acc[64 * j + h + 3]), 0.f), s);
+          }
+        }
+        if (j == 0 && sub == 0 && lane == 0 && it < 16) CSA_T(tslot, 48 + it);
+        if (e < (j == 0 ? nvis0 : nvis1)) {
+          if constexpr (kFuse)
+            sSlice[e - t_begin * kTileE] = s;
+          else
+            p.scores[static_cast<size_t>(q + j) * p.E_stride + e] = s;
+          if (p.score_out) p.score_out[static_cast<size_t>(q + j) * p.E_max + e] = s;
+        }
       }
     }
   }
@@ -393,7 +437,7 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT>::kThreads, 2)
   CSA_TB(3);
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, Shape::kTmem);
   }
   if constexpr (kFuse) {
     // ---------------------------------------------------------------- selection
@@ -797,7 +841,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 }
 
-int g_index_smem[5][64];
+int g_index_smem[6][64];
 
 }  // namespace
 
@@ -808,7 +852,9 @@ size_t index_workspace_bytes(int Nq, int E_max, int /*k*/) {
 
 cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s) {
   const int row_bytes = a.Di / 2;
-  const int N = std::max(16, (a.Hi + 15) / 16 * 16);
+  const bool grouped = a.q_group == 2;
+  if (grouped && (a.Hi != 64 || a.Di != 128 || a.q_raw != nullptr)) return cudaErrorInvalidValue;
+  const int N = grouped ? 128 : std::max(16, (a.Hi + 15) / 16 * 16);  // B rows: one query's heads, or a pair's
   CUtensorMap tm_k, tm_q;
   const CUtensorMapSwizzle swz = row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   if (!encode_2d_u8(&tm_k, a.k_fp4, row_bytes, static_cast<uint64_t>(a.B) * a.E_max, row_bytes, kTileE, swz))
@@ -829,8 +875,13 @@ cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s) {
   p.E_stride = a.E_stride;
   p.N = N;
   const int tiles_max = (a.E_max + kTileE - 1) / kTileE;
-  int splits = std::max(1, std::min(tiles_max, 2 * num_sms() / std::max(1, a.Nq)));
-  splits = std::max(splits, (tiles_max + kMaxTilesPerCta - 1) / kMaxTilesPerCta);
+  // splits of each query's (group's) entry range: about one wave of CTAs, and no CTA
+  // with more tiles than it stages scale bytes for
+  const int units = grouped ? (a.Nq + 1) / 2 : a.Nq;
+  const int per_sm = grouped ? 1 : 2;
+  const int max_tiles = grouped ? kQMaxTiles : kMaxTilesPerCta;
+  int splits = std::max(1, std::min(tiles_max, per_sm * num_sms() / std::max(1, units)));
+  splits = std::max(splits, (tiles_max + max_tiles - 1) / max_tiles);
   p.tiles_per_cta = (tiles_max + splits - 1) / splits;
   p.splits = (tiles_max + p.tiles_per_cta - 1) / p.tiles_per_cta;
   p.w = a.w;
@@ -842,6 +893,15 @@ cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s) {
   p.scores = a.scores_ws;
   p.score_out = a.score_out;
   p.err = device_error_word();
+
+  if (grouped) {  // pairs of queries of one sequence share every key tile
+    constexpr size_t smem = IndexShape<0, 8, 2>::kSmem;
+    const cudaError_t e =
+        set_dyn_smem(reinterpret_cast<const void*>(index_score_kernel<64, false, 0, 8, 2>), smem, g_index_smem[5]);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(index_score_kernel<64, false, 0, 8, 2>, dim3(units * p.splits), dim3(kIdxThreads), smem, s,
+                      tm_k, tm_q, p);
+  }
 
   // many pre-encoded queries of the common shape: persistent CTAs, several queries each
   if (a.q_raw == nullptr && a.Hi == 64 && a.Di == 128 && a.Nq >= 2 * num_sms() &&
@@ -906,7 +966,7 @@ bool index_topk_fusable(int Nq, int Hi, int Di, int E_max, int k, bool raw_q, in
 cudaError_t launch_index_topk_fused(const IndexArgs& a, cudaStream_t s, bool* launched) {
   *launched = false;
   int C = 0, ept = 0;
-  if (a.idx_out == nullptr || a.cnt_out == nullptr ||
+  if (a.idx_out == nullptr || a.cnt_out == nullptr || a.q_group == 2 ||
       !index_topk_fusable(a.Nq, a.Hi, a.Di, a.E_max, a.k, a.q_raw != nullptr, &C, &ept))
     return cudaSuccess;
   CUtensorMap tm_k, tm_q;

@@ -130,6 +130,7 @@ struct IndexArgs {
   float* score_out;  // nullable
   float* scores_ws;  // [Nq, E_stride]
   int E_stride;
+  int q_group;       // 2: rows 2g, 2g+1 share a sequence and every key tile (Hi = 64, Di = 128); else 1
 };
 size_t index_workspace_bytes(int Nq, int E_max, int k);
 cudaError_t launch_index_score(const IndexArgs& a, cudaStream_t s);  // writes scores_ws (+ score_out)
@@ -170,6 +171,9 @@ struct AttnArgs {
   float* lse;
   void* ws;
   size_t ws_bytes;
+  int q_prep;               // 1: q is raw; the kernel applies RMSNorm (q_norm) + partial RoPE
+  int q_norm, rope_dims;
+  float q_eps, rope_theta;
 };
 size_t attn_workspace_bytes(int Nq, int H, int D, int max_keys);
 // Batch-invariant attention (process-wide, off by default): a query's key list is split

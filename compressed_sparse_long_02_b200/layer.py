@@ -5,11 +5,11 @@ rabbit", CSA / window / indexer paragraphs):
     csa_compress(kv)            -> entries (norm + RoPE) and raw window rows
     csa_compress(indexer keys)  -> MXFP4 indexer key cache
     csa_quantize_mxfp4(q_I)     -> MXFP4 indexer queries
-    csa_norm_rope(q)            -> attention queries
     csa_index_topk              -> top-k entry indices per query
-    csa_sparse_attn             -> output
-CSA decode: csa_quantize_mxfp4(q_I) -> csa_index_topk (scores and selection in one
-fused kernel at decode shapes) -> csa_sparse_attn over a resident cache.  HCA prefill: csa_compress(m'=128) -> csa_norm_rope(q) -> hca_attn.
+    csa_sparse_attn_ex          -> output (the queries' RMSNorm + RoPE applied as the
+                                   kernel loads them, bitwise csa_norm_rope's)
+CSA decode: csa_quantize_mxfp4(q_I) -> csa_index_topk -> csa_sparse_attn over a resident
+cache.  HCA prefill: csa_compress(m'=128) -> hca_attn_ex.
 """
 from __future__ import annotations
 
@@ -17,11 +17,16 @@ import torch
 
 from . import binding as B
 
-__all__ = ["csa_prefill", "csa_decode", "hca_prefill"]
+__all__ = ["csa_prefill", "csa_decode", "hca_prefill", "q_prep"]
 
 
 def _i32(x, dev):
     return torch.as_tensor(x, dtype=torch.int32, device=dev)
+
+
+def q_prep(wl) -> dict:
+    """The queries' RMSNorm + partial RoPE, applied by the attention kernel as it loads them."""
+    return dict(norm=wl.norm, eps=wl.eps, rope_dims=wl.rope_dims, theta=wl.theta)
 
 
 def csa_prefill(wl, t: dict, rows: torch.Tensor | None = None) -> dict:
@@ -38,15 +43,14 @@ def csa_prefill(wl, t: dict, rows: torch.Tensor | None = None) -> dict:
     Nq = pos.numel()
     qi = t["qi"][0] if rows is None else t["qi"][0][rows]
     q_fp4, q_sc = B.csa_quantize_mxfp4(qi)
-    qraw = t["q"][0] if rows is None else t["q"][0][rows]
-    q = B.csa_norm_rope(qraw, pos, norm=wl.norm, eps=wl.eps, rope_dims=wl.rope_dims, theta=wl.theta)
+    q = (t["q"][0] if rows is None else t["q"][0][rows]).contiguous()  # raw: prepared inside the attention
     w = (t["w"][0] if rows is None else t["w"][0][rows]).contiguous()
     seq = torch.zeros(Nq, dtype=torch.int32, device=dev)
     n_ent = _i32([E], dev)
     idx, cnt, _ = B.csa_index_topk(q_fp4, q_sc, w, pos, seq, keys["fp4"], keys["fp4_scale"], n_ent, k=wl.k,
                                    m=wl.m)
     out, lse = B.csa_sparse_attn(q, pos, seq, pool["entries"], idx, cnt, pool["window"], _i32([0], dev), W=wl.W,
-                                 want_lse=True)
+                                 want_lse=True, prep=q_prep(wl))
     return dict(out=out, lse=lse, idx=idx, cnt=cnt, entries=pool["entries"], window=pool["window"],
                 k_fp4=keys["fp4"], k_scale=keys["fp4_scale"], q=q, q_fp4=q_fp4, q_scale=q_sc, w=w, n_ent=n_ent)
 
@@ -83,9 +87,8 @@ def hca_prefill(wl, t: dict, rows: torch.Tensor | None = None) -> dict:
                           rope_dims=wl.rope_dims, theta=wl.theta, want_window=True)
     E = T // wl.m
     pos = torch.arange(T, dtype=torch.int32, device=dev) if rows is None else rows.to(torch.int32)
-    qraw = t["q"][0] if rows is None else t["q"][0][rows]
-    q = B.csa_norm_rope(qraw, pos, norm=wl.norm, eps=wl.eps, rope_dims=wl.rope_dims, theta=wl.theta)
+    q = (t["q"][0] if rows is None else t["q"][0][rows]).contiguous()  # raw: prepared inside the attention
     seq = torch.zeros(pos.numel(), dtype=torch.int32, device=dev)
     out, lse = B.hca_attn(q, pos, seq, pool["entries"], _i32([E], dev), pool["window"], _i32([0], dev),
-                          mprime=wl.m, W=wl.W, want_lse=True)
+                          mprime=wl.m, W=wl.W, want_lse=True, prep=q_prep(wl))
     return dict(out=out, lse=lse, entries=pool["entries"], window=pool["window"], q=q)

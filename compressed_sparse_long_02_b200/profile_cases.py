@@ -11,8 +11,8 @@ counters mean something, and a few GB on the device at most):
   norm_rope_q_2k    csa_norm_rope of 2048 query rows x 64 heads x 512 (bf16)
   quantize_qi_8k    csa_quantize_mxfp4 of 8192 x 64 x 128 bf16 indexer queries
   decode_128k       the 128K decode step's indexer, top-k and attention calls (32 queries)
-  attn_csa_4k       csa_sparse_attn of 4096 prefill queries (k=512, W=128) over 1024 entries
-  attn_hca_8k       hca_attn of 8192 prefill queries over 64 entries + the 128-token window
+  attn_csa_4k       csa_sparse_attn_ex of 4096 raw prefill queries (k=512, W=128) over 1024 entries
+  attn_hca_8k       hca_attn_ex of 8192 raw prefill queries over 64 entries + the 128-token window
   proj_2k           csa_grouped_out_proj of 2048 tokens (64 heads of 512, 8 groups, R=1024, 4096)
 """
 from __future__ import annotations
@@ -69,10 +69,10 @@ def run(case: str, reps: int) -> None:
         ne = torch.tensor([wl.E], dtype=torch.int32, device=dev)
         if wl.kind == "csa_prefill":
             fn = lambda: B.csa_sparse_attn(r["q"], pos, seq, r["entries"], r["idx"], r["cnt"], r["window"], zero,
-                                           W=wl.W, out=r["out"])
+                                           W=wl.W, out=r["out"], prep=layer.q_prep(wl))
         else:
             fn = lambda: B.hca_attn(r["q"], pos, seq, r["entries"], ne, r["window"], zero, mprime=wl.m, W=wl.W,
-                                    out=r["out"])
+                                    out=r["out"], prep=layer.q_prep(wl))
     elif case == "proj_2k":
         ps = synth.PROJ["csa_prefill_8k"]
         d = synth.proj_inputs_torch(ps, dev, T=2048)

@@ -12,9 +12,11 @@
  *   csa_compress_step   the same for decode: the entry a new token completes.
  *   csa_norm_rope       RMSNorm + partial RoPE of query heads (and raw window rows).
  *   csa_quantize_mxfp4  FP4 (E2M1, UE8M0 scale per 32) encoding for the lightning indexer.
- *   csa_index_topk      lightning-indexer scores of every visible entry, then top-k.
+ *   csa_index_topk      lightning-indexer scores of every visible entry, then top-k
+ *                       (csa_index_topk_grouped: queries of one sequence share the key reads).
  *   csa_sparse_attn     shared-KV MQA over the top-k entries plus the raw-token window.
  *   hca_attn            shared-KV MQA over every visible HCA entry plus the window.
+ *   csa_sparse_attn_ex, hca_attn_ex  the same with the query's RMSNorm + RoPE applied in the kernel.
  *   csa_grouped_out_proj  grouped projection of the head outputs to the hidden size.
  *
  * Conventions shared by every call
@@ -192,6 +194,26 @@ CSA_API csa_status csa_index_topk(int Nq, int Hi, int Di, int k, int m, const ui
                           int32_t* cnt_out, float* score_out, void* workspace, size_t ws_bytes,
                           cudaStream_t stream);
 CSA_API size_t csa_index_topk_workspace(int Nq, int E_max, int k);
+
+/*
+ * csa_index_topk_grouped -- csa_index_topk for multi-query decode: several new tokens of
+ * one sequence scored together (multi-token-prediction drafts: "DeepSeek-V4: Towards Highly
+ * Efficient Million-Token Context Intelligence", section 2, keeps V3's multi-token
+ * prediction).  Query rows come in groups of q_group consecutive
+ * rows that name the same sequence; every key tile is read once per group and one
+ * N = q_group x 64 block-scaled MMA scores all of the group's heads.  Outputs are bitwise
+ * those of csa_index_topk on the same rows.
+ * Supported: q_group 1 (exactly csa_index_topk) or 2 with Hi = 64 and Di = 128; Nq may
+ * be odd (the last group has one row).  A group row that names another sequence than
+ * the group's first row records CSA_DEVERR_INDEX and scores -inf for every entry
+ * visible to it.  Same workspace as csa_index_topk.
+ */
+CSA_API csa_status csa_index_topk_grouped(int q_group, int Nq, int Hi, int Di, int k, int m, const uint8_t* q_fp4,
+                                          const uint8_t* q_scale, const float* w, const int32_t* q_pos,
+                                          const int32_t* q_seq, int B, int E_max, const uint8_t* k_fp4,
+                                          const uint8_t* k_scale, const int32_t* n_entries, int32_t* idx_out,
+                                          int32_t* cnt_out, float* score_out, void* workspace, size_t ws_bytes,
+                                          cudaStream_t stream);
 /* Kernels csa_index_topk launches for these sizes (pre-encoded queries): 1 when the fused
  * decode kernel runs, 2 otherwise (the scoring kernel, then the top-k kernel), 0 for
  * Nq < 1.  See csa_set_index_fusion. */
@@ -299,6 +321,37 @@ CSA_API csa_status hca_attn(int Nq, int H, int D, int mprime, int W, float scale
                     const int32_t* n_entries, int Tw, const void* window_kv, const int32_t* window_base,
                     void* out, float* lse, void* workspace, size_t ws_bytes, cudaStream_t stream);
 CSA_API size_t hca_attn_workspace(int Nq, int H, int D, int E_max, int W);
+
+/*
+ * Query preparation inside the attention kernels: csa_sparse_attn_ex and hca_attn_ex
+ * take the RAW query q (bf16 [Nq, H, D]) and apply the transform of csa_norm_rope
+ * (dtype bf16, pos = q_pos) to every head row: RMSNorm with unit gain when norm != 0,
+ * then the partial RoPE on the last rope_dims channels.  The kernel rotates those
+ * channels in place and folds each head's norm into its logit scale (a rotation commutes
+ * with a scale), so the result equals csa_norm_rope followed by csa_sparse_attn /
+ * hca_attn up to rounding, without the extra pass over q in HBM.  Supported: rope_dims
+ * even, 0 <= rope_dims <= 64.
+ */
+typedef struct {
+  int norm;         /* 1: RMSNorm (unit gain) of each head row */
+  float eps;        /* RMSNorm epsilon */
+  int rope_dims;    /* partial RoPE on the last rope_dims channels (0 = none) */
+  float rope_theta; /* RoPE base */
+} csa_q_prep;
+
+/* As csa_sparse_attn / hca_attn, with q raw and prepared in the kernel as `prep` says
+ * (prep NULL: q is used as given, i.e. the plain calls).  Same workspace sizes.
+ * Errors: as the plain calls; UNSUPPORTED for rope_dims odd, negative or above 64. */
+CSA_API csa_status csa_sparse_attn_ex(const csa_q_prep* prep, int Nq, int H, int D, int k, int W, float scale,
+                                      const void* q, const int32_t* q_pos, const int32_t* q_seq, int B, int E_max,
+                                      const void* entries, const int32_t* idx, const int32_t* cnt, int Tw,
+                                      const void* window_kv, const int32_t* window_base, void* out, float* lse,
+                                      void* workspace, size_t ws_bytes, cudaStream_t stream);
+CSA_API csa_status hca_attn_ex(const csa_q_prep* prep, int Nq, int H, int D, int mprime, int W, float scale,
+                               const void* q, const int32_t* q_pos, const int32_t* q_seq, int B, int E_max,
+                               const void* entries, const int32_t* n_entries, int Tw, const void* window_kv,
+                               const int32_t* window_base, void* out, float* lse, void* workspace, size_t ws_bytes,
+                               cudaStream_t stream);
 
 /*
  * csa_grouped_out_proj -- grouped output projection of the core-attention outputs back to

@@ -82,7 +82,8 @@ def test_decode_calls_reproduce_prefill_bitwise(B, cuda):
     scores = B.csa_index_score(r["q_fp4"][sel].contiguous(), r["q_scale"][sel].contiguous(), r["w"][sel].contiguous(),
                                pos, seq, r["k_fp4"], r["k_scale"], r["n_ent"], m=wl.m)
     idx, cnt = B.csa_topk_select(scores, pos, seq, r["n_ent"], k=wl.k, m=wl.m, E_max=r["k_fp4"].shape[1])
-    out, _ = B.csa_sparse_attn(r["q"][sel].contiguous(), pos, seq, r["entries"], idx, cnt, r["window"], zero, W=wl.W)
+    out, _ = B.csa_sparse_attn(r["q"][sel].contiguous(), pos, seq, r["entries"], idx, cnt, r["window"], zero, W=wl.W,
+                               prep=layer.q_prep(wl))
     assert torch.equal(idx, r["idx"][sel]) and torch.equal(cnt, r["cnt"][sel])
     assert torch.equal(_bits(out), _bits(r["out"][sel])), "decode calls differ from the prefill's rows"
     # and the prefill computed with the mode on is right on those rows

@@ -10,6 +10,7 @@ import math
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 from compressed_sparse_long_02_b200 import synth
@@ -305,6 +306,104 @@ def test_hca_attn_matches_oracle(B, cuda):
     assert_close_attn(t2np(out), ref, "hca attention")
     np.testing.assert_allclose(t2np(lse), lse_ref, atol=2e-2)
     _err_clear(B)
+
+
+@pytest.mark.parametrize("dense", [False, True])
+def test_attn_tile_aligned_boxes_match_oracle(B, cuda, dense):
+    """One CTA per query (>= 148 queries): the key list is tile-aligned where that adds no
+    tile, and full tiles of contiguous rows (dense entries, window rows) load as TMA boxes.
+    Two sequences with their own entry counts and window bases, so that the box row
+    coordinates carry the sequence offsets; queries with full, ragged and padded tiles."""
+    rng = np.random.default_rng(31 + dense)
+    D, H, m, W, E_max, Tw, k = 512, 64, 4, 128, 300, 1200, 256
+    ent = synth.to_dtype_np(rng.standard_normal((2, E_max, D)), "bf16")
+    win = synth.to_dtype_np(rng.standard_normal((2, Tw, D)), "bf16")
+    wbase = np.array([0, 5000], np.int64)
+    ne = np.array([300, 260], np.int32)
+    p0 = np.concatenate([[0, 126, 127, 128, 511, 512, 515, 1023, 1024, 1199], rng.choice(Tw, 90, replace=False)])
+    p1 = np.concatenate([[5000, 5126, 5127, 6199], 5000 + rng.choice(Tw, 96, replace=False)])
+    pos = np.concatenate([np.unique(p0), np.unique(p1)]).astype(np.int64)
+    seq = np.concatenate([np.zeros(len(np.unique(p0)), np.int32), np.ones(len(np.unique(p1)), np.int32)])
+    Nq = len(pos)
+    assert Nq >= 148
+    q = synth.to_dtype_np(rng.standard_normal((Nq, H, D)) * 0.3, "bf16")
+    if dense:
+        idx, cnt = oracle.hca_select(pos, seq, ne, m)
+    else:
+        n_vis = np.minimum((pos + 1) // m, ne[seq]).astype(np.int32)
+        idx = np.full((Nq, k), -1, np.int32)
+        cnt = np.zeros(Nq, np.int32)
+        for i in range(Nq):
+            c = min(k, int(n_vis[i]))
+            idx[i, :c] = np.sort(rng.choice(n_vis[i], c, replace=False)) if c else []
+            cnt[i] = c
+    ref, lse_ref = oracle.attention(q, pos, seq, ent, idx, cnt, win, wbase, W)
+    args = (to_dev_bf16(q, cuda), to_dev(pos.astype(np.int32), cuda), to_dev(seq, cuda), to_dev_bf16(ent, cuda))
+    wb = to_dev(wbase.astype(np.int32), cuda)
+    if dense:
+        out, lse = B.hca_attn(*args, to_dev(ne, cuda), to_dev_bf16(win, cuda), wb, mprime=m, W=W, want_lse=True)
+    else:
+        out, lse = B.csa_sparse_attn(*args, to_dev(idx, cuda), to_dev(cnt, cuda), to_dev_bf16(win, cuda), wb, W=W,
+                                     want_lse=True)
+    assert_close_attn(t2np(out), ref, "tile-aligned attention")
+    np.testing.assert_allclose(t2np(lse), lse_ref, atol=2e-2)
+    _err_clear(B)
+
+
+@pytest.mark.parametrize("dense", [False, True])
+@pytest.mark.parametrize("Nq", [6, 160])
+def test_attn_query_prep_in_kernel(B, cuda, dense, Nq):
+    """csa_sparse_attn_ex / hca_attn_ex on raw queries against the oracle from the raw
+    queries, and against csa_norm_rope followed by the plain call (the same transform,
+    with the norm folded into the logit scale: equal up to rounding).  Few queries (split
+    key lists, two-pass pipeline) and many (one CTA per query, tile boundaries); positions
+    up to 2^20 exercise the angle reduction."""
+    rng = np.random.default_rng(41 + Nq + dense)
+    D, H, m, W, E_max, k = 512, 64, 4, 128, 400, 256
+    Tw = 1 << 20
+    base = Tw - 3000
+    pos = np.sort(rng.choice(np.arange(base, Tw), Nq, replace=False)).astype(np.int64)
+    pos[-1] = Tw - 1
+    seq = np.zeros(Nq, np.int32)
+    ent = synth.to_dtype_np(rng.standard_normal((1, E_max, D)), "bf16")
+    win = synth.to_dtype_np(rng.standard_normal((1, 3000, D)), "bf16")
+    wbase = np.array([base], np.int32)
+    qraw = synth.to_dtype_np(rng.standard_normal((Nq, H, D)) * 2.0, "bf16")
+    idx = np.stack([np.sort(rng.choice(E_max, k, replace=False)) for _ in range(Nq)]).astype(np.int32)
+    cnt = np.full(Nq, k, np.int32)
+    q_d, pos_d, seq_d = to_dev_bf16(qraw, cuda), to_dev(pos.astype(np.int32), cuda), to_dev(seq, cuda)
+    ent_d, win_d, wb_d = to_dev_bf16(ent, cuda), to_dev_bf16(win, cuda), to_dev(wbase, cuda)
+    prep = dict(norm=True, eps=1e-6, rope_dims=64, theta=10000.0)
+    qn = B.csa_norm_rope(q_d, pos_d, norm=True, eps=1e-6, rope_dims=64, theta=10000.0)
+    if dense:
+        ne = to_dev(np.array([E_max], np.int32), cuda)
+        a, la = B.hca_attn(qn, pos_d, seq_d, ent_d, ne, win_d, wb_d, mprime=m, W=W, want_lse=True)
+        b, lb = B.hca_attn_ex(prep, q_d, pos_d, seq_d, ent_d, ne, win_d, wb_d, mprime=m, W=W, want_lse=True)
+    else:
+        idx_d, cnt_d = to_dev(idx, cuda), to_dev(cnt, cuda)
+        a, la = B.csa_sparse_attn(qn, pos_d, seq_d, ent_d, idx_d, cnt_d, win_d, wb_d, W=W, want_lse=True)
+        b, lb = B.csa_sparse_attn_ex(prep, q_d, pos_d, seq_d, ent_d, idx_d, cnt_d, win_d, wb_d, W=W, want_lse=True)
+    torch.cuda.synchronize()
+    assert_close_attn(t2np(b), t2np(a), "in-kernel query prep vs csa_norm_rope + attention")
+    np.testing.assert_allclose(t2np(lb), t2np(la), atol=1e-2)
+    # and against the oracle from the raw queries
+    qf = oracle.prep_queries(qraw, pos, True, 1e-6, 64, 10000.0)
+    if dense:
+        idx, cnt = oracle.hca_select(pos, seq, np.array([E_max]), m)
+    ref, _ = oracle.attention(qf, pos, seq, ent, idx, cnt, win, wbase.astype(np.int64), W)
+    assert_close_attn(t2np(b), ref, "attention with in-kernel query prep")
+    _err_clear(B)
+
+
+def test_attn_query_prep_rejects_unsupported_rope(B, cuda):
+    q = torch.zeros((1, 64, 512), dtype=torch.bfloat16, device=cuda)
+    i1 = torch.zeros(1, dtype=torch.int32, device=cuda)
+    ent = torch.zeros((1, 8, 512), dtype=torch.bfloat16, device=cuda)
+    idx = torch.zeros((1, 4), dtype=torch.int32, device=cuda)
+    for rd in (66, 3, -2):
+        with pytest.raises(B.CsaError):
+            B.csa_sparse_attn_ex(dict(norm=True, eps=1e-6, rope_dims=rd, theta=1e4), q, i1, i1, ent, idx, i1, ent, i1,
+                                 W=4)
 
 
 def test_attn_bad_index_flagged_and_skipped(B, cuda):
