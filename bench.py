@@ -91,12 +91,12 @@ def measure_tensor_peaks(dev, reps: int = 3) -> dict:
 # decode step (profiles/*_decode_128k.md), keyed by the sha1 of the kernel's source file
 # at capture time: a kernel changed since its capture reports traffic null.
 NCU_TRAFFIC = {
-    "attention": {"bytes": 40084736 + 724480, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
-                  "sha1": "eaa29fa8aad8865cf064ea5c1fbdfbb6548616c8"},
-    "index_score": {"bytes": 71479552 + 1724928, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
-                    "sha1": "765ad86bbe490ed1a125c7e5bff8b126b3b9a484"},
-    "topk_select": {"bytes": 4252672, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",
-                    "sha1": "a2d57f7f3c5bef183b3959e4a1cf4ac3611c4eaa"},
+    "attention": {"bytes": 40060928 + 747264, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
+                  "sha1": "ce4e61d6c330e5eb6187025c99670ca421b10950"},
+    "index_score": {"bytes": 71482624 + 1615360, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
+                    "sha1": "0c2280718efcf0aeab21607ede96354751fc5492"},
+    "topk_select": {"bytes": 4253440, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",
+                    "sha1": "cbcd7529cd244ced27564ee5ab128126c7a370bd"},
 }
 
 
