@@ -91,8 +91,8 @@ def measure_tensor_peaks(dev, reps: int = 3) -> dict:
 # decode step (profiles/*_decode_128k.md), keyed by the sha1 of the kernel's source file
 # at capture time: a kernel changed since its capture reports traffic null.
 NCU_TRAFFIC = {
-    "attention": {"bytes": 40060928 + 747264, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
-                  "sha1": "ce4e61d6c330e5eb6187025c99670ca421b10950"},
+    "attention": {"bytes": 40092672 + 604416, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
+                  "sha1": "aa525280d7d7412fcef225d195ef7a0ebd48037a"},
     "index_score": {"bytes": 71482624 + 1615360, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
                     "sha1": "0c2280718efcf0aeab21607ede96354751fc5492"},
     "topk_select": {"bytes": 4253440, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",

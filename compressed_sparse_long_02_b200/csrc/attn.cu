@@ -13,28 +13,25 @@
 //   O^T[512 d, 64 heads]    += V^T[512 x 128] . P^T         (V^T read MN-major, P^T MN-major)
 // with K = V (shared KV).
 //
-// Pipeline.  A tile's 128 rows are gathered slab by slab (a slab = 64 of the 512 dims
-// x 128 rows = 16 KB, SWIZZLE_128B) into a ring of kRing slabs, in the order the MMA
-// warp consumes them:  K0 | K1 V0 | K2 V1 | ... | V(n-1).  The K pass of a tile reads
-// its rows from HBM; the V pass gathers the same rows again (now in L2) once the
-// tile's probabilities exist, so the ring never has to hold a whole tile and QK of tile
-// i+1 runs while the softmax works on tile i.  S^T is double-buffered in TMEM (2 x 64
-// columns), P in shared memory (2 x 16 KB); O^T takes 4 x 64 TMEM columns.
+// A tile's 128 rows arrive slab by slab (a slab = 64 of the 512 dims x 128 rows = 16 KB,
+// SWIZZLE_128B), gathered with cp.async or, for a contiguous run of rows, as a TMA box.
+// Two pipelines:
+//   * attend (shares longer than three tiles: prefill) keeps a tile resident: its eight
+//     slabs fill eight slots (the ring and the first two P buffers), QK reads them, the
+//     softmax writes P into the third P buffer, and PV reads the same slots as V, each
+//     128-dim chunk then releasing its two slots to the next tile -- every key row is
+//     loaded once.  The softmax keeps a running max that only moves when a tile raises it
+//     by more than 2^8 (then O^T is rescaled in TMEM).
+//   * attend_2pass (at most three tiles: decode splits) streams every tile's K slabs from
+//     HBM through a 9-slot ring with S^T of each tile kept in TMEM, runs one exact
+//     softmax, then re-gathers the rows (now in L2) for PV.
+// S^T takes 64 TMEM columns per tile buffer, O^T 4 x 64.  (At M = 128, N = 64 heads a QK
+// MMA of K = 16 costs ~75 cycles and a PV MMA ~64: about half the bf16 rate, whatever the
+// pipeline; loading each row once measured 7 % faster than re-reading it for PV.)
 //
-// Softmax: one thread per (key row, 32 heads); the running max only moves when a tile
-// raises it by more than 2^8 (then O^T is rescaled in TMEM); sums over keys stay per
-// thread and are reduced once at the end.
-//
-// Longer shares (prefill) run tile-resident: a tile's eight slabs fill eight slots (the ring
-// and the first two P buffers), QK reads them, the softmax writes P into the third P
-// buffer, and PV reads the same slots as V, each 128-dim chunk then releasing its two
-// slots to the next tile's loads -- every key row crosses from L2 once.  (At M = 128,
-// N = 64 heads a QK MMA (K = 16) costs ~75 cycles and a PV MMA ~64, about half the bf16
-// rate, and their shared-memory operand reads compete with the slab loads; reading each
-// row once measured 7 % faster than streaming the V pass again.)
-//
-// Roles (416 threads): warps 0-7 softmax + epilogue, warps 8-11 gather producers
-// (cp.async, 16-byte chunks; Q arrives by TMA), warp 12 TMEM owner and MMA issuer.
+// Roles (416 threads): warps 0-7 softmax + epilogue, warps 8-11 producers (cp.async
+// gathers of 16-byte chunks, TMA boxes; Q arrives by TMA), warp 12 TMEM owner and MMA
+// issuer.  Sums over keys stay per thread and are reduced once at the end.
 // With one CTA per query the window starts on a tile boundary (when that adds no tile),
 // so a full tile of HCA entries or of window rows is one contiguous run of 128 rows: its
 // slabs arrive as 2-D TMA boxes instead of row gathers.
@@ -77,7 +74,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kSplitSMs = 148;             // B200 SM count used to size decode splits
 constexpr int kMaxSplits = 8;              // portable cluster size
 
-constexpr int kPBufs = 3;           // P buffers: 2 used by the interleaved pipeline, 3 by the two-pass one
+constexpr int kPBufs = 3;           // P buffers: the two-pass pipeline uses 3; attend holds slabs in 2 and P in the third
 constexpr int kMaxTiles2 = kPBufs;  // tiles a CTA's share may have on the two-pass pipeline
 constexpr uint32_t kColO2 = 256;    // two-pass: S^T of up to 3 tiles in [0, 192), O^T in [256, 512)
 // Two-pass slab slots: the K pass cycles through the ring and the P buffers (the softmax
@@ -120,7 +117,6 @@ struct AttnParams {
   float2* part_ml; // [Nq, splits, H]
   int rows_per_split, splits;
   int two_pass;    // every CTA's share is at most kMaxTiles2 tiles: attend_2pass
-  int resident;    // attend: a tile stays in shared memory for its V pass (one load per key row)
   int align;       // tile-aligned key list: the window starts on a tile boundary
   int tma_e;       // dense mode, entries tensor map valid: full entry tiles load by TMA
   int tma_w;       // window tensor map valid: full window tiles load by TMA
@@ -252,24 +248,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
-// Stage st of the slab sequence K0 | K1 V0 | K2 V1 | ... | V(n-1): tile and pass.
-__device__ __forceinline__ void stage_of(int st, int n_tiles, int& tile, bool& is_v) {
-  if (st == 0) {
-    tile = 0;
-    is_v = false;
-  } else if (st == 2 * n_tiles - 1) {
-    tile = n_tiles - 1;
-    is_v = true;
-  } else if (st & 1) {
-    tile = (st + 1) >> 1;
-    is_v = false;
-  } else {
-    tile = (st >> 1) - 1;
-    is_v = true;
-  }
-}
-
 
 // Shared-memory layout of a CTA (one definition for the set-up and the pipeline).
 struct AttnSmem {
@@ -480,27 +458,22 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     };
     bool ok = true;
     int j = 0;  // slab sequence number
-    // resident: only the K pass loads, tile t's slab ka into slot ka (the ring and the
-    // first two P buffers: eight contiguous 16 KB slots), phase t & 1
-    const int n_stages = p.resident ? n_tiles : 2 * n_tiles;
-    for (int st = 0; ok && st < n_stages; ++st) {
-      int tile = st;
-      bool is_v = false;
-      if (!p.resident) stage_of(st, n_tiles, tile, is_v);
-      const uint16_t* src_row = row_src(tile, !is_v);
+    // tile t's slab ka goes into slot ka (the ring and the first two P buffers: eight
+    // contiguous 16 KB slots), phase t & 1
+    for (int tile = 0; ok && tile < n_tiles; ++tile) {
+      const uint16_t* src_row = row_src(tile, true);
       const bool valid = src_row != nullptr;
       const uint16_t* src = valid ? src_row : p.entries;
       const unsigned long long src_ll = reinterpret_cast<unsigned long long>(src);
       const TileBox box = tile_box(p, kl, tm_e, tm_w, row_begin + tile * kBN, row_end);
       for (int ka = 0; ka < kSlabs; ++ka, ++j) {
-        const int slot = p.resident ? ka : j % kRing;
-        const uint32_t use = p.resident ? static_cast<uint32_t>(tile) : static_cast<uint32_t>(j / kRing);
-        if (!warp_wait(&slot_free[slot], (use & 1) ^ 1, p.err, abort_flag)) {
+        const int slot = ka;
+        if (!warp_wait(&slot_free[slot], (tile & 1) ^ 1, p.err, abort_flag)) {
           ok = false;
           break;
         }
         if (ptid == 0 && tslot == 4 && j < 64) CSA_T(10, j);
-        if (!is_v && ka == 0 && lane < nrows) {
+        if (ka == 0 && lane < nrows) {
           // the softmax of the tile two back (same buffer) finished before this slot freed
           row_ok[(tile & 1) * 128 + r0 + lane] = valid ? 1 : 0;
           mbar_arrive(&row_ready[tile & 1]);
@@ -544,9 +517,9 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     const int rope_atom = p.q_prep && p.rope_dims > 0 ? (kD - p.rope_dims) / 64 : kSlabs;
     bool q_ready_seen = rope_atom >= kSlabs;
     int j = 0;
-    // resident: QK(t) from slots 0..7, then (once P(t) is written) PV(t) from the same slots,
-    // each 128-dim chunk releasing its two slots to tile t + 1; P in the third P buffer
-    for (int tile = 0; ok && p.resident && tile < n_tiles; ++tile) {
+    // QK(t) from slots 0..7, then (once P(t) is written) PV(t) from the same slots, each
+    // 128-dim chunk releasing its two slots to tile t + 1; P in the third P buffer
+    for (int tile = 0; ok && tile < n_tiles; ++tile) {
       const int b = tile & 1;
       if (tile >= 2 && !warp_wait(&s_free[b], ((tile - 2) >> 1) & 1, p.err, abort_flag)) break;
       for (int ka = 0; ka < kSlabs; ++ka, ++j) {
@@ -595,79 +568,6 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
         if (tile < 8) CSA_T(tslot, 32 + tile);
       }
       __syncwarp();
-    }
-    for (int st = 0; ok && !p.resident && st < 2 * n_tiles; ++st) {
-      int tile;
-      bool is_v;
-      stage_of(st, n_tiles, tile, is_v);
-      const int b = tile & 1;
-      if (!is_v) {
-        // S^T[b] = K Q^T slab by slab; buffer b was last read by the softmax of tile - 2
-        if (tile >= 2 && !warp_wait(&s_free[b], ((tile - 2) >> 1) & 1, p.err, abort_flag)) break;
-        for (int ka = 0; ka < kSlabs; ++ka, ++j) {
-          const int slot = j % kRing;
-          if (!warp_wait(&full[slot], (j / kRing) & 1, p.err, abort_flag)) {
-            ok = false;
-            break;
-          }
-          if (!q_ready_seen && ka >= rope_atom) {  // the query's rotated channels are written
-            q_ready_seen = true;
-            if (!warp_wait(L.q_ready, 0, p.err, abort_flag)) {
-              ok = false;
-              break;
-            }
-          }
-          if (lane == 0 && tslot == 4 && j < 64) CSA_T(12, j);
-          fence_proxy_async_smem();  // the producers' cp.async writes, seen through the barrier
-          tc_fence_after();
-          if (lane == 0) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(tmem + kColS + 64 * b,
-                       smem_desc(ring0 + slot * kSlabBytes + kk * 32, 16, 1024, kSwizzle128B),
-                       smem_desc(q0 + ka * 8192 + kk * 32, 16, 1024, kSwizzle128B), idesc_qk, (ka | kk) ? 1u : 0u);
-            tc_commit(&slot_free[slot]);
-          }
-          __syncwarp();
-        }
-        if (!ok) break;
-        if (lane == 0) {
-          tc_commit(&s_full[b]);
-          if (tile < 8) CSA_T(tslot, 24 + tile);
-        }
-        __syncwarp();
-      } else {
-        // O^T += V^T P^T[b], one 128-dim chunk (two adjacent ring slots) at a time
-        if (!warp_wait(&p_full[b], (tile >> 1) & 1, p.err, abort_flag)) break;
-        tc_fence_after();
-        for (int dc = 0; dc < 4; ++dc, j += 2) {
-          const int slot = j % kRing;  // j even and kRing even: slot + 1 is the chunk's second slab
-          if (!warp_wait(&full[slot], (j / kRing) & 1, p.err, abort_flag) ||
-              !warp_wait(&full[slot + 1], ((j + 1) / kRing) & 1, p.err, abort_flag)) {
-            ok = false;
-            break;
-          }
-          fence_proxy_async_smem();
-          tc_fence_after();
-          if (lane == 0) {
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-              mma_bf16(tmem + kColO + 64 * dc,
-                       smem_desc(ring0 + slot * kSlabBytes + ks * 2048, kSlabBytes, 1024, kSwizzle128B),
-                       smem_desc(p0 + b * 16384 + ks * 2048, 16384, 1024, kSwizzle128B), idesc_pv,
-                       (tile > 0 || ks > 0) ? 1u : 0u);
-            tc_commit(&slot_free[slot]);
-            tc_commit(&slot_free[slot + 1]);
-          }
-          __syncwarp();
-        }
-        if (!ok) break;
-        if (lane == 0) {
-          tc_commit(o_done);
-          if (tile < 8) CSA_T(tslot, 32 + tile);
-        }
-        __syncwarp();
-      }
     }
     // o_done may have two phases outstanding when the softmax finishes its last tile, so
     // the epilogue waits on a barrier of its own
@@ -778,9 +678,9 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
       float (&pr)[32] = x;
       // P[b] was last read by PV of tile it - 2, which completed before QK of this tile
       // signalled s_full (one thread issues both, and a commit covers every earlier MMA)
-      // (resident: the third buffer, last read by PV of tile it - 1, which also completed
-      // before QK of this tile signalled s_full)
-      uint8_t* pb = sP + (p.resident ? 2 : b) * 16384;
+      // P in the third buffer, last read by PV of tile it - 1, which completed before QK of
+      // this tile signalled s_full (one thread issues both; a commit covers every earlier MMA)
+      uint8_t* pb = sP + 2 * 16384;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const uint4 w4 = make_uint4(pack_bf16x2(pr[8 * c], pr[8 * c + 1]), pack_bf16x2(pr[8 * c + 2], pr[8 * c + 3]),
@@ -1516,7 +1416,6 @@ cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s) {
   const int rows = p.align ? pad_keys : max_keys;
   p.rows_per_split = std::max(32, (((rows + splits - 1) / splits) + 31) / 32 * 32);
   p.two_pass = p.rows_per_split <= kMaxTiles2 * kBN ? 1 : 0;
-  p.resident = p.two_pass ? 0 : 1;
   if (static_cast<int64_t>(a.Nq) * kH >= INT32_MAX) return cudaErrorInvalidValue;  // 32-bit TMA row coordinate
   CUtensorMap tm_q;  // the queries as 64-row x 128-byte boxes
   if (!encode_2d_u8(&tm_q, a.q, kD * 2, static_cast<uint64_t>(a.Nq) * kH, 128, kH, CU_TENSOR_MAP_SWIZZLE_128B))
