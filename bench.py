@@ -253,6 +253,9 @@ DECODE_CALLS = ["quantize", "index_topk", "attention"]
 # 128K decode, 71 us device step, 3.15 MB up and 2 MB down per step at ~50 GB/s each
 # way): 2 sets 300K, 3 sets 393K, 4 sets 440K queries/s against 459K on the device alone
 E2E_BUFFERS = 4
+# steps of the end-to-end measurement (host wall clock around the pipelined steps): at
+# ~70 us a step, the default 20 would time ~1.4 ms, where one host hiccup moves the figure
+E2E_MIN_STEPS = 400
 
 
 def decode_step(wl, cache, step, ws, ev=None):
@@ -549,10 +552,11 @@ def bench_decode_e2e(args, wl, caches, steps, ws, dist):
     torch.cuda.synchronize()
     dist.barrier()
     t0 = time.perf_counter()
-    run(0, args.steps)
+    n_steps = max(args.steps, E2E_MIN_STEPS)  # wall-clock timing: long enough that host jitter averages out
+    run(0, n_steps)
     t = dist.max(time.perf_counter() - t0)
     del g_up, g_comp, g_down
-    return {"value": wl.B * dist.world * args.steps / t, "unit": UNIT, "h2d_bytes_per_step": h2d,
+    return {"value": wl.B * dist.world * n_steps / t, "unit": UNIT, "steps": n_steps, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
             "pipelined": "upload of step i+1 and download of step i-1 overlap step i; each stage a CUDA graph replay"}
 

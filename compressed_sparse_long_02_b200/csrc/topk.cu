@@ -285,13 +285,56 @@ __global__ void __launch_bounds__(THREADS) topk_reg_kernel(TopkParams p) {
 
 int g_topk_smem[2][64];
 
+// Whether Nq clusters of 16 CTAs of 1024 threads can be resident at once (a cluster of 16
+// needs 16 free SMs in one GPC); the answer per device is cached.
+bool topk_cluster16_fits(int Nq) {
+  static int max_clusters[64];  // 0: not asked yet, -1: none
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (max_clusters[dev] == 0) {
+    int n = 0;
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(topk_reg_kernel<16, 1024, 16>),
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(16);
+      cfg.blockDim = dim3(1024);
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 16;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(topk_reg_kernel<16, 1024, 16>), &cfg) !=
+          cudaSuccess)
+        n = 0;
+    }
+    cudaGetLastError();  // a refused query leaves no sticky error
+    max_clusters[dev] = n > 0 ? n : -1;
+  }
+  return max_clusters[dev] >= Nq;
+}
+
 // one cluster of C CTAs (1024 threads each) per row, the fewest entries per thread that hold the row
 template <int C>
 cudaError_t launch_topk_cluster(const TopkParams& t, int Nq, int E_max, cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>(Nq * C)), block(1024);
+  if constexpr (C == 16) {  // a non-portable cluster size: rows of up to 16 x 1024 x 16 entries
+    static int allowed[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !allowed[dev]) {
+      const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(topk_reg_kernel<16, 1024, 16>),
+                                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+      allowed[dev] = 1;
+    }
+    return launch_pdl_cluster(topk_reg_kernel<16, 1024, 16>, grid, block, 0, C, s, t);
+  } else {
   if (E_max <= C * 1024 * 8) return launch_pdl_cluster(topk_reg_kernel<C, 1024, 8>, grid, block, 0, C, s, t);
   if (E_max <= C * 1024 * 16) return launch_pdl_cluster(topk_reg_kernel<C, 1024, 16>, grid, block, 0, C, s, t);
   return launch_pdl_cluster(topk_reg_kernel<C, 1024, 32>, grid, block, 0, C, s, t);
+  }
 }
 
 }  // namespace
@@ -313,10 +356,18 @@ cudaError_t launch_topk_select(const IndexArgs& a, cudaStream_t s) {
   // Few rows longer than 2048 entries: a cluster of C CTAs per row, C as large as one wave
   // of CTAs (one per SM) allows and the cluster's registers hold the row.
   int C = 0;
-  if (a.E_max > 2048)
+  if (a.E_max > 2048) {
+    // 16 CTAs (a non-portable cluster) only for rows beyond 8 x 1024 x 16 entries (the
+    // 1M-context decode), and only where 16-CTA clusters can be resident at once
+    if (a.E_max > 8 * 1024 * 16 && a.E_max <= 16 * 1024 * 16 && static_cast<int64_t>(a.Nq) * 16 <= num_sms() &&
+        topk_cluster16_fits(a.Nq))
+      C = 16;
     for (int c = 8; c >= 2 && C == 0; c >>= 1)
       if (static_cast<int64_t>(a.Nq) * c <= num_sms() && static_cast<int64_t>(c) * 1024 * 32 >= a.E_max) C = c;
-  if (C == 8) {
+  }
+  if (C == 16) {
+    e = launch_topk_cluster<16>(t, a.Nq, a.E_max, s);
+  } else if (C == 8) {
     e = launch_topk_cluster<8>(t, a.Nq, a.E_max, s);
   } else if (C == 4) {
     e = launch_topk_cluster<4>(t, a.Nq, a.E_max, s);

@@ -202,7 +202,8 @@ template <int C, int THREADS, int EPT>
 __device__ __forceinline__ void topk_regs_row(const TopkParams& p, int row, int rank, const float (&v)[EPT],
                                               TopkMask<EPT> valid) {
   static_assert(EPT == 8 || EPT == 16 || EPT == 32 || EPT == 64, "EPT: 8, 16, 32 or 64 entries per thread");
-  static_assert(C >= 1 && C <= 8, "portable cluster sizes");
+  static_assert(C == 1 || C == 2 || C == 4 || C == 8 || C == 16, "cluster sizes: 1 to 8 (portable) or 16");
+  constexpr int kRedLanes = C > 8 ? 16 : 8;  // lanes of warp 0 holding one CTA's value each
   static_assert(THREADS * EPT <= 32768, "a CTA's count in one bin fits 16 bits");
   using Mask = TopkMask<EPT>;
   constexpr Mask kOne = 1;
@@ -285,7 +286,7 @@ __device__ __forceinline__ void topk_regs_row(const TopkParams& p, int row, int 
     lo = __uint_as_float(rg[0]);
     hi = __uint_as_float(rg[1]);
 #pragma unroll
-    for (int o = 4; o > 0; o >>= 1) {  // C <= 8 lanes
+    for (int o = kRedLanes / 2; o > 0; o >>= 1) {
       lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
       hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
@@ -351,11 +352,11 @@ __device__ __forceinline__ void topk_regs_row(const TopkParams& p, int row, int 
     const uint32_t nc = lane < C ? cta_word<C>(&s_ncand, lane) : 0u;
     uint32_t incl = nc;
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
+    for (int o = 1; o < kRedLanes; o <<= 1) {
       const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    const uint32_t total = __shfl_sync(0xffffffffu, incl, 7);
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, kRedLanes - 1);
     if (total <= 32u) {
       // lane j < total fetches the j-th member key (CTAs in order), then the warp ranks them
       uint32_t key = 0;
@@ -461,7 +462,7 @@ __device__ __forceinline__ void topk_regs_row(const TopkParams& p, int row, int 
       if (lane < rank) cta_words<C, 2>(s_cnt, lane, gq);
       uint32_t g = gq[0], q = gq[1];
 #pragma unroll
-      for (int o = 4; o > 0; o >>= 1) {  // C <= 8 lanes
+      for (int o = kRedLanes / 2; o > 0; o >>= 1) {
         g += __shfl_xor_sync(0xffffffffu, g, o);
         q += __shfl_xor_sync(0xffffffffu, q, o);
       }

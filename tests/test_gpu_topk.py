@@ -2,8 +2,8 @@
 
 The same float32 score rows go to both sides, so index sets must be identical (no tie
 exemption: ties resolve to the lowest index on both sides).  Cases span every kernel
-variant -- rows held in the registers of a thread-block cluster of 2, 4 or 8 CTAs (few
-rows: 8, 16 or 32 entries per thread), of one CTA (many rows: 16 / 32 entries per
+variant -- rows held in the registers of a thread-block cluster of 2, 4, 8 or 16 CTAs
+(few rows: 8, 16 or 32 entries per thread), of one CTA (many rows: 16 / 32 entries per
 thread, rows up to 2048, 8192 and 32768 entries), and rows staged in shared memory
 (longer rows, read from global memory beyond its capacity) -- with ragged visible
 counts, rows at or below k, exact ties across warp and CTA boundaries, -0/+0, negative
@@ -91,6 +91,23 @@ def test_topk_cluster_of_eight(B, cuda, Nq, E):
     s[0, E // 8 - 700:E // 8 + 700] = 6.5     # a tie group across the first CTA boundary
     n_vis = np.full(Nq, E, np.int32)
     n_vis[-1] = E - 12345
+    _run(B, cuda, s, n_vis, k, E)
+
+
+@pytest.mark.parametrize("Nq,E", [(4, 262144), (9, 150000)])
+@pytest.mark.parametrize("kind", ["normal", "levels", "outlier", "equal"])
+def test_topk_cluster_of_sixteen(B, cuda, Nq, E, kind):
+    """Rows beyond 131072 entries with at most 9 rows: a non-portable cluster of 16 CTAs per
+    row, 16 entries per thread, where 16-CTA clusters can be resident (else 8 CTAs of 32);
+    a tie group across the first CTA boundary, ragged visible counts."""
+    rng = np.random.default_rng(500 + Nq + len(kind))
+    k = 1024
+    s = _rows(kind, Nq, E, rng)
+    if kind == "normal":
+        s[0, E // 16 - 900:E // 16 + 900] = 6.5
+    n_vis = np.full(Nq, E, np.int32)
+    n_vis[-1] = E - 54321
+    n_vis[1] = k + 1
     _run(B, cuda, s, n_vis, k, E)
 
 
