@@ -170,6 +170,87 @@ __device__ void cluster_select_bin(const uint32_t* h, uint32_t need, uint32_t* s
   __syncthreads();
 }
 
+// The same search for large clusters (C >= 8) as a reduce-scatter: CTA r owns the bins
+// [r NB / C, (r + 1) NB / C), sums only those over the cluster into s_own (one 32-bit count
+// per bin) and publishes their total in *s_owntot; after one cluster barrier every CTA
+// finds the owner of the need-th largest key from the C totals (ranked from the top bin,
+// which CTA C - 1 owns) and scans that owner's bins.  A CTA reads 2 NB / C + NB / C words
+// of distributed shared memory instead of C NB / 2 (for C = 16 and NB = 4096: 1.5 KB per
+// thread block instead of 128 KB), at the price of that barrier.  The caller has
+// synchronised the cluster after the histograms were complete; s_own and *s_owntot are
+// rewritten only after the next such barrier.
+template <int C, int THREADS, int NB>
+__device__ void cluster_select_bin_rs(const uint32_t* h, uint32_t need, int rank, uint32_t* s_bin, uint32_t* s_above,
+                                      uint32_t* warp_buf, uint32_t* s_tot, uint32_t* s_own, uint32_t* s_owntot,
+                                      uint32_t* s_sel) {
+  constexpr int OWN = NB / C;   // bins a CTA owns
+  constexpr int OWNW = OWN / 2;  // their words
+  static_assert(C >= 2 && C <= 32 && NB % (2 * C) == 0 && OWNW <= THREADS, "owned words: one per thread at most");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t mine = 0;
+  if (static_cast<int>(threadIdx.x) < OWNW) {
+    const uint32_t* w = h + rank * OWNW + threadIdx.x;
+    uint32_t x[C];
+#pragma unroll
+    for (int r = 0; r < C; ++r) x[r] = cta_word<C>(w, r);  // all in flight at once
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int r = 0; r < C; ++r) {
+      lo += x[r] & 0xFFFFu;
+      hi += x[r] >> 16;
+    }
+    s_own[2 * threadIdx.x] = lo;
+    s_own[2 * threadIdx.x + 1] = hi;
+    mine = lo + hi;
+  }
+  block_excl_scan<THREADS>(mine, warp_buf, s_tot);
+  if (threadIdx.x == 0) *s_owntot = *s_tot;
+  cta_group_sync<C>();  // every CTA's owned sums and total are published
+  if (warp == 0) {
+    const uint32_t t = lane < C ? cta_word<C>(s_owntot, lane) : 0u;
+    uint32_t suf = t;  // inclusive suffix sum over lanes (CTA C - 1 owns the top bins)
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
+      if (lane + o < 32) suf += y;
+    }
+    const uint32_t above_r = suf - t;
+    const uint32_t who = __ballot_sync(0xffffffffu, lane < C && above_r < need && need <= suf);
+    const int owner = who ? __ffs(who) - 1 : 0;
+    if (lane == owner) {
+      s_sel[0] = static_cast<uint32_t>(owner);
+      s_sel[1] = above_r;
+    }
+  }
+  __syncthreads();
+  const int owner = static_cast<int>(s_sel[0]);
+  const uint32_t base = s_sel[1];
+  // the owner's bins from the top: thread t takes [OWN - (t + 1) PER, OWN - t PER)
+  constexpr int PER = (OWN + THREADS - 1) / THREADS;
+  const int lo_bin = OWN - PER * (static_cast<int>(threadIdx.x) + 1);
+  uint32_t c[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) c[i] = lo_bin + i >= 0 ? cta_word<C>(s_own + lo_bin + i, owner) : 0u;
+  uint32_t local = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) local += c[i];
+  const uint32_t pre = base + block_excl_scan<THREADS>(local, warp_buf, s_tot);
+  if (pre < need && need <= pre + local) {
+    uint32_t acc = pre;
+    bool found = false;
+#pragma unroll
+    for (int i = PER - 1; i >= 0; --i) {
+      if (!found && acc + c[i] >= need) {
+        *s_bin = static_cast<uint32_t>(owner * OWN + lo_bin + i);
+        *s_above = acc;
+        found = true;
+      }
+      acc += c[i];
+    }
+  }
+  __syncthreads();
+}
+
 // add one key to bin b of a histogram of 16-bit counts, two per word
 __device__ __forceinline__ void hist16_add(uint32_t* h, uint32_t b) { atomicAdd(&h[b >> 1], 1u << ((b & 1u) << 4)); }
 
@@ -219,6 +300,8 @@ __device__ __forceinline__ void topk_regs_row(const TopkParams& p, int row, int 
   __shared__ float s_grange[2];            // the row's
   __shared__ uint32_t s_cand[32];          // this CTA's first 32 member keys
   __shared__ uint32_t s_thr[2];
+  // reduce-scatter search (C >= 8): this CTA's owned bin sums, their total, the owner found
+  __shared__ uint32_t s_own[C >= 8 ? kBins / C : 1], s_owntot, s_sel[2];
   __shared__ __align__(8) uint32_t s_cnt[2];  // this CTA's kept counts: above the threshold, equal to it
   __shared__ uint32_t s_cbase[2];          // the same summed over the CTAs before this one
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -317,7 +400,11 @@ __device__ __forceinline__ void topk_regs_row(const TopkParams& p, int row, int 
   CSA_T(tslot, 8);
   cta_group_sync<C>();  // every CTA's counts are complete
   CSA_T(tslot, 9);
-  cluster_select_bin<C, THREADS, kBins>(hist[0], static_cast<uint32_t>(p.k), &s_bin, &s_above, warp_buf, &s_tot);
+  if constexpr (C >= 8)
+    cluster_select_bin_rs<C, THREADS, kBins>(hist[0], static_cast<uint32_t>(p.k), rank, &s_bin, &s_above, warp_buf,
+                                             &s_tot, s_own, &s_owntot, s_sel);
+  else
+    cluster_select_bin<C, THREADS, kBins>(hist[0], static_cast<uint32_t>(p.k), &s_bin, &s_above, warp_buf, &s_tot);
   const uint32_t b1 = s_bin;
   const uint32_t above1 = s_above;
   CSA_T(tslot, 2);
@@ -405,7 +492,11 @@ __device__ __forceinline__ void topk_regs_row(const TopkParams& p, int row, int 
         }
       }
       cta_group_sync<C>();
-      cluster_select_bin<C, THREADS, NB>(h, need - above, &s_bin, &s_above, warp_buf, &s_tot);
+      if constexpr (C >= 8)
+        cluster_select_bin_rs<C, THREADS, NB>(h, need - above, rank, &s_bin, &s_above, warp_buf, &s_tot, s_own,
+                                              &s_owntot, s_sel);
+      else
+        cluster_select_bin<C, THREADS, NB>(h, need - above, &s_bin, &s_above, warp_buf, &s_tot);
       prefix = (prefix << kWidth) | s_bin;
       above += s_above;
       __syncthreads();
