@@ -91,7 +91,7 @@ constexpr size_t kOffP = kOffRing + kRing * kSlabBytes;           // kPBufs x 16
 constexpr size_t kOffSmall = kOffP + kPBufs * 16384;              // reductions, stats, barriers
 // reductions and stats (832 floats), rope table (32 float2), row flags, 40 barriers, TMEM
 // slot and abort flag, laid out by AttnSmem below
-constexpr size_t kSmallUsed = 832 * 4 + 32 * 8 + 128 * kPBufs + (1 + 2 * kSlotBars + kPBufs + 2 + 2 + 1 + kPBufs + 2) * 8 + 8;
+constexpr size_t kSmallUsed = 832 * 4 + 32 * 8 + 128 * kPBufs + (1 + 2 * kSlotBars + kPBufs + 2 + 2 + 1 + kPBufs + 4) * 8 + 8;
 constexpr size_t kOffIdx = kOffSmall + 5120;                      // this CTA's slice of the index list
 static_assert(kSmallUsed <= 5120, "small shared-memory region");
 constexpr int kIdxCap = 2048;
@@ -117,6 +117,7 @@ struct AttnParams {
   float2* part_ml; // [Nq, splits, H]
   int rows_per_split, splits;
   int two_pass;    // every CTA's share is at most kMaxTiles2 tiles: attend_2pass
+  int persist;     // splits == 1 and attend: persistent CTAs take queries blockIdx.x, + gridDim.x, ...
   int align;       // tile-aligned key list: the window starts on a tile boundary
   int tma_e;       // dense mode, entries tensor map valid: full entry tiles load by TMA
   int tma_w;       // window tensor map valid: full window tiles load by TMA
@@ -273,6 +274,9 @@ struct AttnSmem {
   uint64_t* row_ready;  // [kPBufs] producers: row_ok of a tile written
   uint64_t* fin;        // MMA commit: every MMA of the CTA complete
   uint64_t* q_ready;    // softmax warps: the query prepared in place (query preparation only)
+  uint64_t* q_free;     // Q's slabs may be reloaded: the query's last QK completed (MMA commit) and
+                        // the softmax threads read Q for the last time (query preparation)
+  uint64_t* o_free;     // softmax warps: O^T of a query read from TMEM (the next query may overwrite it)
   uint32_t* tmem_slot;
   volatile int* abort_flag;
   int32_t* sidx;        // this CTA's slice of the index list
@@ -300,7 +304,9 @@ struct AttnSmem {
     row_ready = o_done + 1;
     fin = row_ready + kPBufs;
     q_ready = fin + 1;
-    tmem_slot = reinterpret_cast<uint32_t*>(q_ready + 1);
+    q_free = q_ready + 1;
+    o_free = q_free + 1;
+    tmem_slot = reinterpret_cast<uint32_t*>(o_free + 1);
     abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);
   }
@@ -320,7 +326,7 @@ struct AttnSmem {
 // quarter c = t % 4): in the last atom, chunks 2c and 2c + 1 of row h (16 channels); for
 // the norm, 112 channels of atoms 0..6 plus those 16.  cs_tab holds the (cos, sin) of the
 // query's rope pairs; ssq the per-thread sums of squares of the raw last-atom channels.
-__device__ __forceinline__ void prep_query(const AttnParams& p, int n, uint8_t* sQ, uint64_t* q_full,
+__device__ __forceinline__ void prep_query(const AttnParams& p, int n, uint8_t* sQ, uint64_t* q_full, uint32_t q_ph,
                                            uint64_t* q_ready, float* hscale, float2* cs_tab,
                                            volatile int* abort_flag, int warp, int lane) {
   const int t = static_cast<int>(threadIdx.x);  // 0..255 (softmax warps)
@@ -329,7 +335,7 @@ __device__ __forceinline__ void prep_query(const AttnParams& p, int n, uint8_t* 
   const int rope_base = kD - p.rope_dims;  // >= 448: inside the last atom
   if (warp == 0 && lane < npairs)  // overlaps the query's load
     cs_tab[lane] = rowprep::rope_cs(static_cast<double>(p.q_pos[n]), rowprep::inv_freq(p.rope_theta, lane, p.rope_dims));
-  const bool got = warp_wait(q_full, 0, p.err, abort_flag);
+  const bool got = warp_wait(q_full, q_ph, p.err, abort_flag);
   named_bar_sync(1, 256);  // cs_tab written
   float ss = 0.f;
   if (got) {
@@ -388,9 +394,14 @@ __device__ __forceinline__ void prep_query(const AttnParams& p, int n, uint8_t* 
 
 // One CTA's share of a query: rows [row_begin, row_end) of its key list, n_tiles > 0.
 // Writes the normalised output (splits == 1) or the unnormalised partial + (max, sum).
+// A CTA may take several queries in turn (persistent CTAs): qi counts the queries this CTA
+// took before this one, T0 their tiles, so that every barrier's phase continues; the
+// roles do not wait for one another between queries (the next query's loads and QK run
+// while the softmax warps write this one's output).
 __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& tm_q, const CUtensorMap& tm_e,
                                        const CUtensorMap& tm_w, uint8_t* smem, uint32_t tmem, int n, int split,
-                                       const KeyList& kl, int row_begin, int row_end, int n_tiles) {
+                                       const KeyList& kl, int row_begin, int row_end, int n_tiles, int qi,
+                                       int T0) {
   const AttnSmem L(smem);
   uint8_t* sQ = L.sQ;
   uint8_t* sRing = L.sRing;
@@ -428,13 +439,15 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     const int ptid = threadIdx.x - 256;
     const int r0 = kRowsPerProd * pw;
     const int nrows = min(kRowsPerProd, kBN - r0);
-    if (ptid == 0) {
-      // query: 64 head rows x 1 KB as 8 boxes of 64 rows x 128 B (one per 64-dim atom)
+    // query: 64 head rows x 1 KB as 8 boxes of 64 rows x 128 B (one per 64-dim atom), once
+    // the previous query's last QK has released Q's slabs
+    if (ptid == 0 && (qi == 0 || mbar_wait(L.q_free, (qi - 1) & 1, p.err, abort_flag))) {
       mbar_arrive_expect_tx(q_full, kH * kD * 2);
       for (int a = 0; a < 8; ++a) tma_load_2d(smem_u32(sQ + a * 8192), &tm_q, q_full, 128 * a, n * kH);
     }
     // this CTA's slice of the index list, staged once per warp (no dependent global load
-    // per row); each warp copies the part its own lanes will read
+    // per row); each warp copies the part its own lanes will read (they finished reading
+    // the previous query's slice: their last gathers were issued)
     const int sel_here = max(0, min(row_end, kl.n_sel) - row_begin);
     const bool staged = !p.dense && sel_here <= kIdxCap;
     if (staged)
@@ -466,17 +479,18 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
       const uint16_t* src = valid ? src_row : p.entries;
       const unsigned long long src_ll = reinterpret_cast<unsigned long long>(src);
       const TileBox box = tile_box(p, kl, tm_e, tm_w, row_begin + tile * kBN, row_end);
+      const int T = T0 + tile;  // the CTA's tile count: phases continue across its queries
       for (int ka = 0; ka < kSlabs; ++ka, ++j) {
         const int slot = ka;
-        if (!warp_wait(&slot_free[slot], (tile & 1) ^ 1, p.err, abort_flag)) {
+        if (!warp_wait(&slot_free[slot], (T & 1) ^ 1, p.err, abort_flag)) {
           ok = false;
           break;
         }
         if (ptid == 0 && tslot == 4 && j < 64) CSA_T(10, j);
         if (ka == 0 && lane < nrows) {
           // the softmax of the tile two back (same buffer) finished before this slot freed
-          row_ok[(tile & 1) * 128 + r0 + lane] = valid ? 1 : 0;
-          mbar_arrive(&row_ready[tile & 1]);
+          row_ok[(T & 1) * 128 + r0 + lane] = valid ? 1 : 0;
+          mbar_arrive(&row_ready[T & 1]);
           if (ptid == 0 && tile < 8) CSA_T(tslot, 8 + tile);
         }
         const uint32_t dst = smem_u32(sRing + slot * kSlabBytes);
@@ -505,14 +519,14 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     cp_async_wait_all();  // nothing in flight when the CTA exits
     {  // Q must have landed before the CTA may exit (already true on the normal path)
       volatile int never = 0;
-      if (ptid == 0) mbar_wait(q_full, 0, p.err, &never);
+      if (ptid == 0) mbar_wait(q_full, qi & 1, p.err, &never);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_qk = idesc_bf16(128, kH, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16(128, kH, true, true);
     const uint32_t q0 = smem_u32(sQ), ring0 = smem_u32(sRing), p0 = smem_u32(sP);
-    bool ok = warp_wait(q_full, 0, p.err, abort_flag);
+    bool ok = warp_wait(q_full, qi & 1, p.err, abort_flag);
     // query preparation: the rotated atoms are ready for the MMA once q_ready completes
     const int rope_atom = p.q_prep && p.rope_dims > 0 ? (kD - p.rope_dims) / 64 : kSlabs;
     bool q_ready_seen = rope_atom >= kSlabs;
@@ -520,16 +534,17 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     // QK(t) from slots 0..7, then (once P(t) is written) PV(t) from the same slots, each
     // 128-dim chunk releasing its two slots to tile t + 1; P in the third P buffer
     for (int tile = 0; ok && tile < n_tiles; ++tile) {
-      const int b = tile & 1;
-      if (tile >= 2 && !warp_wait(&s_free[b], ((tile - 2) >> 1) & 1, p.err, abort_flag)) break;
+      const int T = T0 + tile;
+      const int b = T & 1;
+      if (T >= 2 && !warp_wait(&s_free[b], ((T - 2) >> 1) & 1, p.err, abort_flag)) break;
       for (int ka = 0; ka < kSlabs; ++ka, ++j) {
-        if (!warp_wait(&full[ka], tile & 1, p.err, abort_flag)) {
+        if (!warp_wait(&full[ka], T & 1, p.err, abort_flag)) {
           ok = false;
           break;
         }
         if (!q_ready_seen && ka >= rope_atom) {  // the query's rotated channels are written
           q_ready_seen = true;
-          if (!warp_wait(L.q_ready, 0, p.err, abort_flag)) {
+          if (!warp_wait(L.q_ready, qi & 1, p.err, abort_flag)) {
             ok = false;
             break;
           }
@@ -548,10 +563,13 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
       if (!ok) break;
       if (lane == 0) {
         tc_commit(&s_full[b]);
+        if (tile == n_tiles - 1) tc_commit(L.q_free);  // Q's slabs are read by no later MMA
         if (tile < 8) CSA_T(tslot, 24 + tile);
       }
       __syncwarp();
-      if (!warp_wait(&p_full[b], (tile >> 1) & 1, p.err, abort_flag)) break;
+      if (!warp_wait(&p_full[b], (T >> 1) & 1, p.err, abort_flag)) break;
+      // the first PV of a query overwrites O^T: the previous query's epilogue must have read it
+      if (tile == 0 && qi > 0 && !warp_wait(L.o_free, (qi - 1) & 1, p.err, abort_flag)) break;
       tc_fence_after();
       if (lane == 0) {
         for (int dc = 0; dc < 4; ++dc) {
@@ -577,10 +595,15 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     // ------------------------------------------------------------ softmax (warps 0-7)
     // thread = one key row of the tile (TMEM lane 32*(warp%4)+lane) and 32 heads
     // (hh = warp/4 selects heads 0-31 or 32-63).
+    if (threadIdx.x < kH) {  // the query's running statistics (the previous query's epilogue is done)
+      m_run[threadIdx.x] = -INFINITY;
+      l_run[threadIdx.x] = 0.f;
+    }
     if (p.q_prep)
-      prep_query(p, n, sQ, q_full, L.q_ready, L.hscale, L.cs_tab, abort_flag, warp, lane);
+      prep_query(p, n, sQ, q_full, qi & 1, L.q_ready, L.hscale, L.cs_tab, abort_flag, warp, lane);
     else if (threadIdx.x < kH)
       L.hscale[threadIdx.x] = p.scale_log2;
+    mbar_arrive(L.q_free);  // this thread reads Q no more (the norm reads are done)
     named_bar_sync(1, 256);
     const float* hscale = L.hscale;
     const int q4 = warp & 3, hh = warp >> 2;
@@ -592,8 +615,9 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     for (int i = 0; i < 32; ++i) lacc[i] = 0.f;
     bool ok = true;
     for (int it = 0; it < n_tiles; ++it) {
-      const int b = it & 1;
-      const uint32_t ph = (it >> 1) & 1;
+      const int T = T0 + it;
+      const int b = T & 1;
+      const uint32_t ph = (T >> 1) & 1;
       const bool got_s = mbar_wait(&s_full[b], ph, p.err, abort_flag);
       if (named_bar_or(1, 256, !got_s)) {
         ok = false;
@@ -690,7 +714,7 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
       if (move_max && it > 0) {
         // move this warp's O^T columns (heads h0..h0+31) to the new max once PV of tile
         // it - 1 is complete (PV of tile it waits for this warp's arrival on p_full)
-        const bool got_o = mbar_wait(o_done, (it - 1) & 1, p.err, abort_flag);
+        const bool got_o = mbar_wait(o_done, (T - 1) & 1, p.err, abort_flag);
         if (named_bar_or(1, 256, !got_o)) {
           ok = false;
           break;
@@ -718,7 +742,7 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     }
     // ------------------------------------------------------------ epilogue
     CSA_TB(6);
-    const bool fin_ok = !named_bar_or(1, 256, !mbar_wait(fin, 0, p.err, abort_flag));  // all 256 take part
+    const bool fin_ok = !named_bar_or(1, 256, !mbar_wait(fin, qi & 1, p.err, abort_flag));  // all 256 take part
     ok = ok && fin_ok;
     CSA_TB(7);
     if (t == 0 && hh == 0) CSA_T(tslot, 2);
@@ -743,6 +767,10 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
           tmem_ld16(ta + 16, o[c] + 16);
         }
         tmem_wait_ld();
+        if (dp == 2) {  // O^T is read: the CTA's next query may overwrite it
+          tc_fence_before();
+          mbar_arrive(L.o_free);
+        }
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int d = (dp + c) * 128 + t;
@@ -771,6 +799,7 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     } else if (threadIdx.x < kH && p.splits > 1) {  // gave up: this split contributes nothing
       p.part_ml[(static_cast<size_t>(n) * p.splits + split) * kH + threadIdx.x] = make_float2(-INFINITY, 0.f);
     }
+    if (!ok) mbar_arrive(L.o_free);  // (ok is the same for all 256 threads)
   }
 
   if (threadIdx.x == 0) CSA_T(tslot, 3);
@@ -993,7 +1022,7 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
     // ------------------------------------------------------------ softmax (warps 0-7)
     // thread = key row t of each tile (TMEM lane 32 (warp % 4) + lane) and 32 heads
     if (p.q_prep)
-      prep_query(p, n, L.sQ, L.q_full, L.q_ready, L.hscale, L.cs_tab, L.abort_flag, warp, lane);
+      prep_query(p, n, L.sQ, L.q_full, 0, L.q_ready, L.hscale, L.cs_tab, L.abort_flag, warp, lane);
     else if (threadIdx.x < kH)
       L.hscale[threadIdx.x] = p.scale_log2;
     named_bar_sync(1, 256);
@@ -1169,6 +1198,8 @@ __device__ __forceinline__ uint32_t attn_setup(uint8_t* smem) {
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(L.q_ready, 256);
+    mbar_init(L.q_free, 257);  // the MMA's commit after the last QK + the 256 softmax threads
+    mbar_init(L.o_free, 256);
     for (int i = 0; i < kSlotBars; ++i) {
       mbar_init(&full[i], kProdThreads);
       mbar_init(&slot_free[i], 1);
@@ -1264,6 +1295,10 @@ __device__ __forceinline__ void merge_partials(const AttnParams& p, int n, int h
   }
 }
 
+// kPersist: persistent CTAs on the tile-resident pipeline (splits == 1); otherwise one query
+// (or one split of a query) per CTA on either pipeline.  Two instantiations, so that each
+// keeps its own register allocation.
+template <bool kPersist>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_e,
                 const __grid_constant__ CUtensorMap tm_w, AttnParams p) {
@@ -1276,9 +1311,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (p.tma_w) prefetch_tmap(&tm_w);
   }
   const uint32_t tmem = attn_setup(smem);
+  if constexpr (kPersist) {
+    // Persistent CTAs (splits == 1 on the tile-resident pipeline) take queries blockIdx.x,
+    // + gridDim.x, ...: the set-up above happens once, and while the softmax warps write one
+    // query's output the producers and the MMA warp already start the next.
+    griddep_enter();
+    CSA_TB(1);
+    const AttnSmem L(smem);
+    int qi = 0, T0 = 0;
+    for (int n = static_cast<int>(blockIdx.x); n < p.Nq; n += static_cast<int>(gridDim.x)) {
+      const KeyMeta meta = key_meta(p, n);
+      if (!meta.ok) {  // a sequence out of range: no output, recorded
+        if (threadIdx.x == 0) atomicExch(p.err, CSA_DEVERR_INDEX);
+        continue;
+      }
+      const KeyList kl = key_list(p, n, meta);
+      const int row_end = min(kl.win0 + kl.n_win, p.rows_per_split);
+      const int n_tiles = row_end > 0 ? (row_end + kBN - 1) / kBN : 0;
+      if (n_tiles == 0) {  // nothing to attend to: the softmax warps write zeros, the rest go on
+        if (threadIdx.x < 256) {
+          for (int i = threadIdx.x; i < kH * kD / 2; i += 256)
+            reinterpret_cast<uint32_t*>(p.out + static_cast<size_t>(n) * kH * kD)[i] = 0u;
+          if (p.lse && threadIdx.x < kH) p.lse[n * kH + threadIdx.x] = -INFINITY;
+        }
+        continue;
+      }
+      attend(p, tm_q, tm_e, tm_w, smem, tmem, n, 0, kl, 0, row_end, n_tiles, qi, T0);
+      ++qi;
+      T0 += n_tiles;
+      if (*L.abort_flag) break;  // a wait gave up: every role leaves (its own waits fail at once)
+    }
+    tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == kMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kTmemCols);
+    }
+    return;
+  }
   const int n = blockIdx.x / p.splits;
   const int split = blockIdx.x % p.splits;  // the CTA's rank in its cluster when splits > 1
-  const KeyMeta meta = key_meta(p, n);
+  const KeyMeta meta = key_meta(p, n);      // before the wait (no kernel of this library writes it)
   griddep_enter();
   CSA_TB(1);
   const bool seq_ok = meta.ok;  // same for every CTA of the query (cluster)
@@ -1292,12 +1365,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     row_end = min(nk, row_begin + p.rows_per_split);
     n_tiles = row_end > row_begin ? (row_end - row_begin + kBN - 1) / kBN : 0;
   }
-
   if (n_tiles > 0) {
     if (p.two_pass)
       attend_2pass(p, tm_q, tm_e, tm_w, smem, tmem, n, split, kl, row_begin, row_end, n_tiles);
     else
-      attend(p, tm_q, tm_e, tm_w, smem, tmem, n, split, kl, row_begin, row_end, n_tiles);
+      attend(p, tm_q, tm_e, tm_w, smem, tmem, n, split, kl, row_begin, row_end, n_tiles, 0, 0);
   }
   tc_fence_before();
   __syncthreads();
@@ -1338,7 +1410,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   CSA_TB(5);
 }
 
-int g_attn_smem[64];
+int g_attn_smem[2][64];
 
 std::atomic<int> g_batch_invariant{0};
 
@@ -1416,6 +1488,7 @@ cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s) {
   const int rows = p.align ? pad_keys : max_keys;
   p.rows_per_split = std::max(32, (((rows + splits - 1) / splits) + 31) / 32 * 32);
   p.two_pass = p.rows_per_split <= kMaxTiles2 * kBN ? 1 : 0;
+  p.persist = (splits == 1 && !p.two_pass) ? 1 : 0;
   if (static_cast<int64_t>(a.Nq) * kH >= INT32_MAX) return cudaErrorInvalidValue;  // 32-bit TMA row coordinate
   CUtensorMap tm_q;  // the queries as 64-row x 128-byte boxes
   if (!encode_2d_u8(&tm_q, a.q, kD * 2, static_cast<uint64_t>(a.Nq) * kH, 128, kH, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -1443,9 +1516,15 @@ cudaError_t launch_attention(const AttnArgs& a, int max_keys, cudaStream_t s) {
     p.part_o = reinterpret_cast<float*>(base);
     p.part_ml = reinterpret_cast<float2*>(base + o_bytes);
   }
-  cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(attn_kernel), kAttnSmem, g_attn_smem);
+  if (p.persist) {
+    cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(attn_kernel<true>), kAttnSmem, g_attn_smem[1]);
+    if (e != cudaSuccess) return e;
+    return launch_pdl_cluster(attn_kernel<true>, dim3(std::min(a.Nq, num_sms())), dim3(kAttnThreads), kAttnSmem, 1u, s,
+                              tm_q, tm_e, tm_w, p);
+  }
+  cudaError_t e = set_dyn_smem(reinterpret_cast<const void*>(attn_kernel<false>), kAttnSmem, g_attn_smem[0]);
   if (e != cudaSuccess) return e;
-  return launch_pdl_cluster(attn_kernel, dim3(a.Nq * splits), dim3(kAttnThreads), kAttnSmem,
+  return launch_pdl_cluster(attn_kernel<false>, dim3(a.Nq * splits), dim3(kAttnThreads), kAttnSmem,
                             static_cast<unsigned>(splits), s, tm_q, tm_e, tm_w, p);
 }
 
