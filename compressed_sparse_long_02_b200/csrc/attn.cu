@@ -62,8 +62,7 @@ constexpr int kSlabs = 8;           // 64-dim slabs per tile
 constexpr int kSlabBytes = 16384;
 constexpr int kRing = 6;            // even: the two slabs of a 128-dim PV chunk sit in adjacent slots
 constexpr int kProdWarps = 4;                          // gather producers
-constexpr int kRowsPerProd = (kBN + kProdWarps - 1) / kProdWarps;  // rows of a tile per producer warp
-static_assert(kRowsPerProd <= 32, "one row per lane");
+static_assert(kBN == 32 * kProdWarps, "one row of a tile per producer lane");
 constexpr int kProdThreads = 32 * kProdWarps;
 constexpr int kMmaWarp = 8 + kProdWarps;               // TMEM owner and MMA issuer
 constexpr int kAttnThreads = 32 * (kMmaWarp + 1);      // 8 softmax warps first
@@ -215,6 +214,58 @@ __device__ __forceinline__ TileBox tile_box(const AttnParams& p, const KeyList& 
 
 __device__ __forceinline__ uint32_t sw128(int row, int chunk) {  // byte offset inside an 8-row x 128 B atom column
   return static_cast<uint32_t>(row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+}
+
+// Row of a tile that lane `l` of gather warp `w` (0-3) owns: a warp takes 32 consecutive
+// rows of the key list (sorted selections put neighbouring entries in one warp's copies),
+// and gather_warp is the owner of a row.
+__device__ __forceinline__ int gather_row(int w, int l) { return 32 * w + l; }
+__device__ __forceinline__ int gather_warp(int row) { return row / 32; }
+
+// Source of row g of query n's key list: a selected entry (g < n_sel), a window row
+// (g >= win0), or nothing (past row_end, the alignment gap, or an index outside the
+// cache, which sets the device error word when `flag`).  `sidx` (nullable) is the CTA's
+// staged slice of the index list, starting at row_begin.
+__device__ __forceinline__ const uint16_t* key_row_src(const AttnParams& p, const KeyList& kl, int n, int g,
+                                                       int row_begin, int row_end, const int32_t* sidx,
+                                                       bool flag) {
+  if (g >= row_end) return nullptr;
+  if (g < kl.n_sel) {
+    const int e = p.dense ? g : (sidx != nullptr ? sidx[g - row_begin] : p.idx[static_cast<size_t>(n) * p.k + g]);
+    if (e >= 0 && e < p.E_max) return p.entries + (static_cast<size_t>(kl.b) * p.E_max + e) * kD;
+    if (flag) atomicExch(p.err, CSA_DEVERR_INDEX);
+    return nullptr;
+  }
+  if (g < kl.win0) return nullptr;
+  const int64_t u = kl.u_lo + (g - kl.win0);
+  return p.window + (static_cast<size_t>(kl.b) * p.Tw + static_cast<size_t>(u - kl.wbase)) * kD;
+}
+
+// Slab ka of a tile (64 dims of its 128 rows) into `dst`, by a group of four warps whose
+// lane l of warp w holds the source of row gather_row(w, l) (src_ll; valid = false: no
+// row, zero-filled): one TMA box when the tile is a contiguous block, else 16-byte
+// cp.async chunks.  Each of the group's 128 threads arrives on `bar` once (the cp.async
+// arrivals when the thread's copies have landed).
+__device__ __forceinline__ void gather_slab(uint32_t dst, const TileBox& box, int ka, unsigned long long src_ll,
+                                            bool valid, int w, int lane, uint64_t* bar) {
+  if (box.map != nullptr) {
+    if (w == 0 && lane == 0) {
+      mbar_arrive_expect_tx(bar, kSlabBytes);
+      tma_load_2d(dst, box.map, bar, ka * 128, box.row);
+    } else {
+      mbar_arrive(bar);
+    }
+    return;
+  }
+#pragma unroll
+  for (int qb = 0; qb < 256; qb += 32) {  // chunk q: 16 bytes q % 8 of the row of lane q / 8
+    const int q = qb + lane;
+    const int rl = q >> 3, c = q & 7;
+    const uint16_t* rs = reinterpret_cast<const uint16_t*>(__shfl_sync(0xffffffffu, src_ll, rl));
+    const bool rv = __shfl_sync(0xffffffffu, valid, rl);
+    cp_async_16(dst + sw128(gather_row(w, rl), c), rs + (ka * 8 + c) * 8, rv);
+  }
+  cp_async_mbar_arrive_noinc(bar);
 }
 
 // 32 per-thread values (one per head) reduced over the 32 lanes of the warp; on return
@@ -432,13 +483,12 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
 
   if (warp >= 8 && warp < 8 + kProdWarps) {
     // ------------------------------------------------------------ gather producers
-    // Producer warp pw owns rows [r0, r0 + nrows) of every tile; each lane resolves one of
-    // them and the warp issues their 8 x 16-byte chunks per slab.  The warps never wait on
-    // one another, so one that gives up cannot stall the others.
+    // Lane l of producer warp pw owns row gather_row(pw, l) of every tile and resolves its
+    // source; the warp issues the 8 x 16-byte chunks per slab of its 32 rows.  The warps
+    // never wait on one another, so one that gives up cannot stall the others.
     const int pw = warp - 8;
     const int ptid = threadIdx.x - 256;
-    const int r0 = kRowsPerProd * pw;
-    const int nrows = min(kRowsPerProd, kBN - r0);
+    const int my_row = gather_row(pw, lane);
     // query: 64 head rows x 1 KB as 8 boxes of 64 rows x 128 B (one per 64-dim atom), once
     // the previous query's last QK has released Q's slabs
     if (ptid == 0 && (qi == 0 || mbar_wait(L.q_free, (qi - 1) & 1, p.err, abort_flag))) {
@@ -452,32 +502,18 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     const bool staged = !p.dense && sel_here <= kIdxCap;
     if (staged)
       for (int i = lane; i < sel_here; i += 32)
-        if ((i % kBN) >= r0 && (i % kBN) < r0 + nrows)
-          sidx[i] = p.idx[static_cast<size_t>(n) * p.k + row_begin + i];
+        if (gather_warp(i % kBN) == pw) sidx[i] = p.idx[static_cast<size_t>(n) * p.k + row_begin + i];
     __syncwarp();
-    // source row of this lane in a tile (nullptr: no row; invalid indices are flagged once)
-    auto row_src = [&](int tile, bool flag) -> const uint16_t* {
-      const int g = row_begin + tile * kBN + r0 + lane;
-      if (lane >= nrows || g >= row_end) return nullptr;
-      if (g < kl.n_sel) {
-        const int e = p.dense ? g : (staged ? sidx[g - row_begin] : p.idx[static_cast<size_t>(n) * p.k + g]);
-        if (e >= 0 && e < p.E_max) return p.entries + (static_cast<size_t>(kl.b) * p.E_max + e) * kD;
-        if (flag) atomicExch(p.err, CSA_DEVERR_INDEX);
-        return nullptr;
-      }
-      if (g < kl.win0) return nullptr;
-      const int64_t u = kl.u_lo + (g - kl.win0);
-      return p.window + (static_cast<size_t>(kl.b) * p.Tw + static_cast<size_t>(u - kl.wbase)) * kD;
-    };
     bool ok = true;
     int j = 0;  // slab sequence number
     // tile t's slab ka goes into slot ka (the ring and the first two P buffers: eight
     // contiguous 16 KB slots), phase t & 1
     for (int tile = 0; ok && tile < n_tiles; ++tile) {
-      const uint16_t* src_row = row_src(tile, true);
+      // source of this lane's row (invalid indices are flagged once)
+      const uint16_t* src_row =
+          key_row_src(p, kl, n, row_begin + tile * kBN + my_row, row_begin, row_end, staged ? sidx : nullptr, true);
       const bool valid = src_row != nullptr;
-      const uint16_t* src = valid ? src_row : p.entries;
-      const unsigned long long src_ll = reinterpret_cast<unsigned long long>(src);
+      const unsigned long long src_ll = reinterpret_cast<unsigned long long>(valid ? src_row : p.entries);
       const TileBox box = tile_box(p, kl, tm_e, tm_w, row_begin + tile * kBN, row_end);
       const int T = T0 + tile;  // the CTA's tile count: phases continue across its queries
       for (int ka = 0; ka < kSlabs; ++ka, ++j) {
@@ -487,33 +523,15 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
           break;
         }
         if (ptid == 0 && tslot == 4 && j < 64) CSA_T(10, j);
-        if (ka == 0 && lane < nrows) {
+        if (ka == 0) {
           // the softmax of the tile two back (same buffer) finished before this slot freed
-          row_ok[(T & 1) * 128 + r0 + lane] = valid ? 1 : 0;
+          row_ok[(T & 1) * 128 + my_row] = valid ? 1 : 0;
           mbar_arrive(&row_ready[T & 1]);
           if (ptid == 0 && tile < 8) CSA_T(tslot, 8 + tile);
         }
-        const uint32_t dst = smem_u32(sRing + slot * kSlabBytes);
-        if (box.map != nullptr) {  // one box per slab; every producer thread still arrives once
-          if (ptid == 0) {
-            mbar_arrive_expect_tx(&full[slot], kSlabBytes);
-            tma_load_2d(dst, box.map, &full[slot], ka * 128, box.row);
-          } else {
-            mbar_arrive(&full[slot]);
-          }
-          continue;
-        }
-        for (int qb = 0; qb < 8 * nrows; qb += 32) {  // warp-uniform trip count: every lane shuffles
-          const int q = qb + lane;                      // chunk q: row r0 + q / 8, 16 bytes q % 8
-          const bool in = q < 8 * nrows;
-          const int rl = in ? q >> 3 : 0, c = q & 7;
-          const uint16_t* rs = reinterpret_cast<const uint16_t*>(__shfl_sync(0xffffffffu, src_ll, rl));
-          const bool rv = __shfl_sync(0xffffffffu, valid, rl);
-          if (in) cp_async_16(dst + sw128(r0 + rl, c), rs + (ka * 8 + c) * 8, rv);
-        }
         // the slab's barrier completes when every producer thread's copies have landed;
         // the consumer fences the async proxy after its wait
-        cp_async_mbar_arrive_noinc(&full[slot]);
+        gather_slab(smem_u32(sRing + slot * kSlabBytes), box, ka, src_ll, valid, pw, lane, &full[slot]);
       }
     }
     cp_async_wait_all();  // nothing in flight when the CTA exits
@@ -859,8 +877,7 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
     // ------------------------------------------------------------ gather producers
     const int pw = warp - 8;
     const int ptid = threadIdx.x - 256;
-    const int r0 = kRowsPerProd * pw;
-    const int nrows = min(kRowsPerProd, kBN - r0);
+    const int my_row = gather_row(pw, lane);
     if (ptid == 0) {
       mbar_arrive_expect_tx(L.q_full, kH * kD * 2);
       for (int a = 0; a < 8; ++a) tma_load_2d(smem_u32(L.sQ + a * 8192), &tm_q, L.q_full, 128 * a, n * kH);
@@ -869,34 +886,22 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
     const bool staged = !p.dense && sel_here <= kIdxCap;
     if (staged)
       for (int i = lane; i < sel_here; i += 32)
-        if ((i % kBN) >= r0 && (i % kBN) < r0 + nrows) L.sidx[i] = p.idx[static_cast<size_t>(n) * p.k + row_begin + i];
+        if (gather_warp(i % kBN) == pw) L.sidx[i] = p.idx[static_cast<size_t>(n) * p.k + row_begin + i];
     __syncwarp();
-    auto row_src = [&](int tile, bool flag) -> const uint16_t* {
-      const int g = row_begin + tile * kBN + r0 + lane;
-      if (lane >= nrows || g >= row_end) return nullptr;
-      if (g < kl.n_sel) {
-        const int e = p.dense ? g : (staged ? L.sidx[g - row_begin] : p.idx[static_cast<size_t>(n) * p.k + g]);
-        if (e >= 0 && e < p.E_max) return p.entries + (static_cast<size_t>(kl.b) * p.E_max + e) * kD;
-        if (flag) atomicExch(p.err, CSA_DEVERR_INDEX);
-        return nullptr;
-      }
-      if (g < kl.win0) return nullptr;
-      const int64_t u = kl.u_lo + (g - kl.win0);
-      return p.window + (static_cast<size_t>(kl.b) * p.Tw + static_cast<size_t>(u - kl.wbase)) * kD;
-    };
     bool ok = true;
     const int nK = kSlabs * n_tiles;
     bool q_free = false;  // the last QK has completed: Q's slabs may take V slabs
     for (int st = 0; ok && st < 2 * n_tiles; ++st) {
       const bool is_v = st >= n_tiles;
       const int tile = is_v ? st - n_tiles : st;
-      const uint16_t* src_row = row_src(tile, !is_v);
+      const uint16_t* src_row = key_row_src(p, kl, n, row_begin + tile * kBN + my_row, row_begin, row_end,
+                                            staged ? L.sidx : nullptr, !is_v);
       const bool valid = src_row != nullptr;
       const unsigned long long src_ll = reinterpret_cast<unsigned long long>(valid ? src_row : p.entries);
       const TileBox box = tile_box(p, kl, tm_e, tm_w, row_begin + tile * kBN, row_end);
       if (ptid == 0) CSA_T(tslot, 8 + st);
-      if (!is_v && lane < nrows) {  // published before this tile's first slab is issued
-        L.row_ok[tile * 128 + r0 + lane] = valid ? 1 : 0;
+      if (!is_v) {  // published before this tile's first slab is issued
+        L.row_ok[tile * 128 + my_row] = valid ? 1 : 0;
         mbar_arrive(&L.row_ready[tile]);
       }
       for (int ka = 0; ka < kSlabs; ++ka) {
@@ -914,25 +919,7 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
           break;
         }
         if (ptid == 0 && tslot == 4 && j < 64) CSA_T(10, j);
-        const uint32_t dst = smem_u32(smem + sl.off);
-        if (box.map != nullptr) {
-          if (ptid == 0) {
-            mbar_arrive_expect_tx(&L.full[sl.bar], kSlabBytes);
-            tma_load_2d(dst, box.map, &L.full[sl.bar], ka * 128, box.row);
-          } else {
-            mbar_arrive(&L.full[sl.bar]);
-          }
-          continue;
-        }
-        for (int qb = 0; qb < 8 * nrows; qb += 32) {
-          const int q = qb + lane;
-          const bool in = q < 8 * nrows;
-          const int rl = in ? q >> 3 : 0, c = q & 7;
-          const uint16_t* rs = reinterpret_cast<const uint16_t*>(__shfl_sync(0xffffffffu, src_ll, rl));
-          const bool rv = __shfl_sync(0xffffffffu, valid, rl);
-          if (in) cp_async_16(dst + sw128(r0 + rl, c), rs + (ka * 8 + c) * 8, rv);
-        }
-        cp_async_mbar_arrive_noinc(&L.full[sl.bar]);
+        gather_slab(smem_u32(smem + sl.off), box, ka, src_ll, valid, pw, lane, &L.full[sl.bar]);
       }
     }
     cp_async_wait_all();
