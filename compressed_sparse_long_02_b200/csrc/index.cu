@@ -10,10 +10,12 @@
 // Score of entry j for query n:  d[h] = <q[n,h], k[j]> (MXFP4 x MXFP4, exact in
 // fp32), S = fp32 chain acc = fmaf(w[n,h], max(d[h],0), acc) over h = 0..Hi-1.
 //
-// index_score_kernel -- one CTA per (query, run of entry tiles).  Entries go on the
-// MMA M axis (128 per tile), the query's heads on N, the head dim on K:
-//   warp 0      TMA producer: key tile 0, the query, the run's key scale bytes (one bulk
-//               copy), then 128 FP4 key rows (SWIZZLE_64B) per stage
+// index_score_kernel -- one CTA per (query, share of its entry tiles): with S CTAs per
+// query, CTA s takes tiles s, s + S, s + 2S, ... (the grouped and fused variants a
+// contiguous run).  Entries go on the MMA M axis (128 per tile), the query's heads on N,
+// the head dim on K:
+//   warp 0      TMA producer: key tile 0, the query, the share's key scale bytes (a bulk
+//               copy per tile), then 128 FP4 key rows (SWIZZLE_64B) per stage
 //   warp 1      TMEM owner and MMA issuer: per tile, one thread tcgen05.cp's the tile's
 //               scale factors into a ring of TMEM slots and issues two
 //               kind::mxf4.block_scale MMAs into one of three accumulators
@@ -179,14 +181,25 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT, kQ>::kThreads, In
   griddep_enter();
   CSA_TB(1);
 
-  // the CTA's first query row (kQ > 1: the group's), and its split of the entry range
+  // the CTA's first query row (kQ > 1: the group's), and its split of the entry tiles:
+  // tiles split, split + splits, split + 2 splits, ... (the query's CTAs stream neighbouring
+  // key tiles at any moment, a few windows of the cache at once rather than one stream
+  // per CTA: measured faster at 128K and 1M); the fused kernel's CTA takes one contiguous
+  // slice (its slice of the scores), and so does the grouped one (measured slower strided)
+  constexpr bool kStrided = !kFuse && kQ == 1;
   const int q = kQ * (kFuse ? static_cast<int>(blockIdx.x) / kFuseC : static_cast<int>(blockIdx.x) / p.splits);
   const int split = kFuse ? static_cast<int>(blockIdx.x) % kFuseC : static_cast<int>(blockIdx.x) % p.splits;
+  const int tiles_per_cta = kFuse ? Shape::kMaxTiles : p.tiles_per_cta;
+  const int tile0 = kStrided ? split : split * tiles_per_cta;  // entry tile of local tile it: tile0 + it * tstride
+  const int tstride = kStrided ? p.splits : 1;
+  auto local_tiles = [&](int nv) {  // this CTA's tiles among the first ceil(nv / 128)
+    const int vt = (nv + kTileE - 1) / kTileE;
+    return vt > tile0 ? min((vt - 1 - tile0) / tstride + 1, tiles_per_cta) : 0;
+  };
   const int seq = p.q_seq[q];
   const bool seq_ok = seq >= 0 && seq < p.B;
   if (!seq_ok && threadIdx.x == 0 && split == 0) atomicExch(p.err, CSA_DEVERR_INDEX);  // produce nothing
   const int nvis0 = seq_ok ? min(visible_entries(p.q_pos[q], p.m, p.n_entries[seq]), p.E_max) : 0;
-  const int tiles_per_cta = kFuse ? Shape::kMaxTiles : p.tiles_per_cta;
   // grouped: the second query row, scored from the same key tiles when it names the same
   // sequence; a row naming another sequence is recorded as an error and gets -inf for
   // every entry visible to it (in this CTA's share), so that its selection is defined
@@ -201,21 +214,22 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT, kQ>::kThreads, In
         nvis1 = nv1;
       } else {
         if (threadIdx.x == 0 && split == 0) atomicExch(p.err, CSA_DEVERR_INDEX);
-        const int e_lo = split * tiles_per_cta * kTileE, e_hi = min(nv1, e_lo + tiles_per_cta * kTileE);
-        for (int e = e_lo + static_cast<int>(threadIdx.x); e < e_hi; e += static_cast<int>(blockDim.x)) {
-          p.scores[static_cast<size_t>(q1) * p.E_stride + e] = -INFINITY;
-          if (p.score_out) p.score_out[static_cast<size_t>(q1) * p.E_max + e] = -INFINITY;
+        const int n1 = local_tiles(nv1);
+        for (int i = static_cast<int>(threadIdx.x); i < n1 * kTileE; i += static_cast<int>(blockDim.x)) {
+          const int e = (tile0 + (i / kTileE) * tstride) * kTileE + i % kTileE;
+          if (e < nv1) {
+            p.scores[static_cast<size_t>(q1) * p.E_stride + e] = -INFINITY;
+            if (p.score_out) p.score_out[static_cast<size_t>(q1) * p.E_max + e] = -INFINITY;
+          }
         }
       }
     }
   }
   const int nvis = max(nvis0, nvis1);
-  const int t_begin = split * tiles_per_cta;
   // fused: a query with at most k visible entries takes all of them (no scoring; the same
   // for every CTA of the cluster, so none reaches a cluster barrier below)
   const bool trivial = kFuse && nvis <= p.k;
-  const int t_end = trivial ? t_begin : min((nvis + kTileE - 1) / kTileE, t_begin + tiles_per_cta);
-  const int n_tiles = t_end - t_begin;  // uniform over the CTA
+  const int n_tiles = trivial ? 0 : local_tiles(nvis);  // uniform over the CTA
 
   const int Hi = kHi > 0 ? kHi : p.Hi;
   const int row_bytes = p.Di / 2;            // 64 (Di=128) or 32 (Di=64)
@@ -232,30 +246,42 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT, kQ>::kThreads, In
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       // key tile 0 first (the long pole), then the query, then every key scale byte of
-      // this CTA's tiles in one bulk copy (they stay in TMEM for the whole run), then the
-      // remaining key tiles as stages free up
-      const int row0 = seq * p.E_max + t_begin * kTileE;
+      // this CTA's tiles (one bulk copy per tile, or one for a contiguous slice; they stay
+      // in TMEM for the whole run), then the remaining key tiles as stages free up
+      const int seq_row = seq * p.E_max;
+      auto tile_e = [&](int it) { return (tile0 + it * tstride) * kTileE; };  // first entry of local tile it
       mbar_arrive_expect_tx(&full[0], a_bytes);
       CSA_T(tslot, 16);
-      tma_load_2d(smem_u32(sA), &tm_k, &full[0], 0, row0);
+      tma_load_2d(smem_u32(sA), &tm_k, &full[0], 0, seq_row + tile_e(0));
       if (!kRawQ) {
         mbar_arrive_expect_tx(b_full, b_bytes);
         tma_load_2d(smem_u32(sB), &tm_q, b_full, 0, q * Hi);
       }
       // entries with a scale byte in the cache: E_max and tile starts are multiples of 8,
-      // so the byte count is a multiple of 16
-      const int sf_entries = min(n_tiles * kTileE, p.E_max - t_begin * kTileE);
-      const uint32_t sf_bytes = static_cast<uint32_t>(sf_entries * sf_row);
-      mbar_arrive_expect_tx(sf_full, sf_bytes);
-      bulk_load(smem_u32(sf_row == 4 ? sSF : sSFraw), p.k_scale + static_cast<size_t>(row0) * sf_row, sf_bytes,
-                sf_full);
+      // so every byte count is a multiple of 16
+      uint8_t* sf_dst = sf_row == 4 ? sSF : sSFraw;
+      const int sf_tile = kTileE * sf_row;  // bytes of a whole tile
+      if (tstride == 1) {
+        const int sf_entries = min(n_tiles * kTileE, p.E_max - tile_e(0));
+        const uint32_t sf_bytes = static_cast<uint32_t>(sf_entries * sf_row);
+        mbar_arrive_expect_tx(sf_full, sf_bytes);
+        bulk_load(smem_u32(sf_dst), p.k_scale + static_cast<size_t>(seq_row + tile_e(0)) * sf_row, sf_bytes, sf_full);
+      } else {
+        const int sf_entries = (n_tiles - 1) * kTileE + min(kTileE, p.E_max - tile_e(n_tiles - 1));
+        mbar_arrive_expect_tx(sf_full, static_cast<uint32_t>(sf_entries * sf_row));
+        for (int it = 0; it < n_tiles; ++it) {
+          const uint32_t bytes = static_cast<uint32_t>(min(kTileE, p.E_max - tile_e(it)) * sf_row);
+          bulk_load(smem_u32(sf_dst + it * sf_tile), p.k_scale + static_cast<size_t>(seq_row + tile_e(it)) * sf_row,
+                    bytes, sf_full);
+        }
+      }
       for (int it = 1; it < n_tiles; ++it) {
         const int st = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
         if (!mbar_wait(&empty[st], ph ^ 1, p.err, abort_flag)) break;
         mbar_arrive_expect_tx(&full[st], a_bytes);
         if (it < 16) CSA_T(tslot, 16 + it);
-        tma_load_2d(smem_u32(sA + st * 8192), &tm_k, &full[st], 0, row0 + it * kTileE);
+        tma_load_2d(smem_u32(sA + st * 8192), &tm_k, &full[st], 0, seq_row + tile_e(it));
       }
     }
   } else if (n_tiles > 0 && warp == 1) {
@@ -405,7 +431,7 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT, kQ>::kThreads, In
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
-      const int e = (t_begin + it) * kTileE + 32 * sub + lane;
+      const int e = (tile0 + it * tstride) * kTileE + 32 * sub + lane;
 #pragma unroll
       for (int j = 0; j < kQ; ++j) {  // query q + j: columns [64 j, 64 j + Hi) of the accumulator
         float s = 0.f;
@@ -422,7 +448,7 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT, kQ>::kThreads, In
         if (j == 0 && sub == 0 && lane == 0 && it < 16) CSA_T(tslot, 48 + it);
         if (e < (j == 0 ? nvis0 : nvis1)) {
           if constexpr (kFuse)
-            sSlice[e - t_begin * kTileE] = s;
+            sSlice[e - tile0 * kTileE] = s;
           else
             p.scores[static_cast<size_t>(q + j) * p.E_stride + e] = s;
           if (p.score_out) p.score_out[static_cast<size_t>(q + j) * p.E_max + e] = s;
@@ -451,9 +477,9 @@ __global__ void __launch_bounds__(IndexShape<kFuseC, kFuseEPT, kQ>::kThreads, In
     }
     // this CTA's slice (written by the epilogue warps before the barrier above) into
     // registers in the layout topk_regs_row takes: v[i] of (warp, lane) is entry
-    // t_begin 128 + 32 kFuseEPT warp + 32 i + lane
+    // tile0 128 + 32 kFuseEPT warp + 32 i + lane
     using Mask = TopkMask<kFuseEPT>;
-    const int e0 = t_begin * kTileE + 32 * kFuseEPT * warp + lane;
+    const int e0 = tile0 * kTileE + 32 * kFuseEPT * warp + lane;
     float v[kFuseEPT];
     Mask valid = 0;
 #pragma unroll
