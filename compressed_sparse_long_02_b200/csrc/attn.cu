@@ -244,16 +244,20 @@ __device__ __forceinline__ const uint16_t* key_row_src(const AttnParams& p, cons
 // Slab ka of a tile (64 dims of its 128 rows) into `dst`, by a group of four warps whose
 // lane l of warp w holds the source of row gather_row(w, l) (src_ll; valid = false: no
 // row, zero-filled): one TMA box when the tile is a contiguous block, else 16-byte
-// cp.async chunks.  Each of the group's 128 threads arrives on `bar` once (the cp.async
-// arrivals when the thread's copies have landed).
+// cp.async chunks.  `bar` takes 128 arrivals per slab: with a box, lane 0 of each warp
+// makes its warp's 32 at once (the first with the byte count); with cp.async, every
+// thread arrives once its own copies have landed.
 __device__ __forceinline__ void gather_slab(uint32_t dst, const TileBox& box, int ka, unsigned long long src_ll,
                                             bool valid, int w, int lane, uint64_t* bar) {
   if (box.map != nullptr) {
-    if (w == 0 && lane == 0) {
-      mbar_arrive_expect_tx(bar, kSlabBytes);
-      tma_load_2d(dst, box.map, bar, ka * 128, box.row);
-    } else {
-      mbar_arrive(bar);
+    if (lane == 0) {
+      if (w == 0) {
+        mbar_arrive_expect_tx(bar, kSlabBytes);
+        tma_load_2d(dst, box.map, bar, ka * 128, box.row);
+        mbar_arrive_cnt(bar, 31);
+      } else {
+        mbar_arrive_cnt(bar, 32);
+      }
     }
     return;
   }
@@ -510,11 +514,11 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
     // contiguous 16 KB slots), phase t & 1
     for (int tile = 0; ok && tile < n_tiles; ++tile) {
       // source of this lane's row (invalid indices are flagged once)
-      const uint16_t* src_row =
-          key_row_src(p, kl, n, row_begin + tile * kBN + my_row, row_begin, row_end, staged ? sidx : nullptr, true);
+      const int ts = row_begin + tile * kBN;
+      const uint16_t* src_row = key_row_src(p, kl, n, ts + my_row, row_begin, row_end, staged ? sidx : nullptr, true);
       const bool valid = src_row != nullptr;
       const unsigned long long src_ll = reinterpret_cast<unsigned long long>(valid ? src_row : p.entries);
-      const TileBox box = tile_box(p, kl, tm_e, tm_w, row_begin + tile * kBN, row_end);
+      const TileBox box = tile_box(p, kl, tm_e, tm_w, ts, row_end);
       const int T = T0 + tile;  // the CTA's tile count: phases continue across its queries
       for (int ka = 0; ka < kSlabs; ++ka, ++j) {
         const int slot = ka;
@@ -710,10 +714,10 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
         const float4 mm = *reinterpret_cast<const float4*>(m_run + h0 + i);
-        x[i] = valid ? exp2f(x[i] - mm.x) : 0.f;
-        x[i + 1] = valid ? exp2f(x[i + 1] - mm.y) : 0.f;
-        x[i + 2] = valid ? exp2f(x[i + 2] - mm.z) : 0.f;
-        x[i + 3] = valid ? exp2f(x[i + 3] - mm.w) : 0.f;
+        x[i] = valid ? fast_exp2(x[i] - mm.x) : 0.f;
+        x[i + 1] = valid ? fast_exp2(x[i + 1] - mm.y) : 0.f;
+        x[i + 2] = valid ? fast_exp2(x[i + 2] - mm.z) : 0.f;
+        x[i + 3] = valid ? fast_exp2(x[i + 3] - mm.w) : 0.f;
       }
 #pragma unroll
       for (int i = 0; i < 32; ++i) lacc[i] += x[i];
