@@ -91,12 +91,12 @@ def measure_tensor_peaks(dev, reps: int = 3) -> dict:
 # decode step (profiles/*_decode_128k.md), keyed by the sha1 of the kernel's source file
 # at capture time: a kernel changed since its capture reports traffic null.
 NCU_TRAFFIC = {
-    "attention": {"bytes": 40092672 + 604416, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
-                  "sha1": "aa525280d7d7412fcef225d195ef7a0ebd48037a"},
-    "index_score": {"bytes": 71482624 + 1615360, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
-                    "sha1": "0c2280718efcf0aeab21607ede96354751fc5492"},
-    "topk_select": {"bytes": 4253440, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",
-                    "sha1": "cbcd7529cd244ced27564ee5ab128126c7a370bd"},
+    "attention": {"bytes": 40103680 + 720640, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
+                  "sha1": "fef08f8a7e38d7502b3cfb83dd239ab69d7d0434"},
+    "index_score": {"bytes": 71483904 + 1665792, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
+                    "sha1": "b271de5f29ab6b90adcc34a460af7ad5b475c231"},
+    "topk_select": {"bytes": 4253184, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",
+                    "sha1": "7fc5928a6f3c6ac7669c341815142304cacfdf34"},
 }
 
 

@@ -13,6 +13,8 @@ counters mean something, and a few GB on the device at most):
   decode_128k       the 128K decode step's indexer, top-k and attention calls (32 queries)
   attn_csa_4k       csa_sparse_attn_ex of 4096 raw prefill queries (k=512, W=128) over 1024 entries
   attn_hca_8k       hca_attn_ex of 8192 raw prefill queries over 64 entries + the 128-token window
+  attn_hca_64k_tail hca_attn_ex of the last 1184 raw queries of a 65536-token prefill (503-512
+                    entries + the window each: the persistent tile-resident path of the 64K layer)
   proj_2k           csa_grouped_out_proj of 2048 tokens (64 heads of 512, 8 groups, R=1024, 4096)
 """
 from __future__ import annotations
@@ -21,7 +23,7 @@ import argparse
 import sys
 
 CASES = ["pool_csa_64k", "pool_hca_64k", "norm_rope_q_2k", "quantize_qi_8k", "decode_128k", "attn_csa_4k",
-         "attn_hca_8k", "proj_2k"]
+         "attn_hca_8k", "attn_hca_64k_tail", "proj_2k"]
 
 
 def run(case: str, reps: int) -> None:
@@ -73,6 +75,22 @@ def run(case: str, reps: int) -> None:
         else:
             fn = lambda: B.hca_attn(r["q"], pos, seq, r["entries"], ne, r["window"], zero, mprime=wl.m, W=wl.W,
                                     out=r["out"], prep=layer.q_prep(wl))
+    elif case == "attn_hca_64k_tail":
+        wl = synth.WORKLOADS["hca_prefill_64k"]
+        n, T, W = 1184, wl.T, wl.W
+        g = torch.Generator(device=dev)
+        g.manual_seed(wl.seed + 7)
+        q = torch.randn((n, wl.H, wl.D), generator=g, device=dev).to(torch.bfloat16)
+        entries = torch.randn((1, wl.E, wl.D), generator=g, device=dev).to(torch.bfloat16)
+        base = T - n - W + 1  # the window buffer holds tokens base .. T - 1
+        window = torch.randn((1, T - base, wl.D), generator=g, device=dev).to(torch.bfloat16)
+        pos = torch.arange(T - n, T, dtype=torch.int32, device=dev)
+        seq = torch.zeros(n, dtype=torch.int32, device=dev)
+        wb = torch.tensor([base], dtype=torch.int32, device=dev)
+        ne = torch.tensor([wl.E], dtype=torch.int32, device=dev)
+        out = torch.empty_like(q)
+        fn = lambda: B.hca_attn(q, pos, seq, entries, ne, window, wb, mprime=wl.m, W=W, out=out,
+                                prep=layer.q_prep(wl))
     elif case == "proj_2k":
         ps = synth.PROJ["csa_prefill_8k"]
         d = synth.proj_inputs_torch(ps, dev, T=2048)
