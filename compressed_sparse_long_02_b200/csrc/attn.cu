@@ -640,27 +640,39 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
       const int T = T0 + it;
       const int b = T & 1;
       const uint32_t ph = (T >> 1) & 1;
-      const bool got_s = mbar_wait(&s_full[b], ph, p.err, abort_flag);
-      if (named_bar_or(1, 256, !got_s)) {
+      // S^T[b] and the tile's row flags; the TMEM load is in flight during the barrier that
+      // agrees on whether both waits succeeded
+      const bool got = mbar_wait(&s_full[b], ph, p.err, abort_flag) && mbar_wait(&row_ready[b], ph, p.err, abort_flag);
+      tc_fence_after();
+      const uint32_t s_addr = tmem + lane_base + kColS + 64 * b + h0;
+      uint32_t sr[32];
+      tmem_ld16(s_addr, sr);
+      tmem_ld16(s_addr + 16, sr + 16);
+      if (named_bar_or(1, 256, !got)) {
+        tmem_wait_ld();
         ok = false;
         break;
       }
       if (t == 0 && hh == 0 && it < 8) CSA_T(tslot, 40 + it);
-      tc_fence_after();
-      const uint32_t s_addr = tmem + lane_base + kColS + 64 * b + h0;
-      const bool got_rows = mbar_wait(&row_ready[b], ph, p.err, abort_flag);
-      if (named_bar_or(1, 256, !got_rows)) {
-        ok = false;
-        break;
-      }
       const bool valid = row_begin + it * kBN + t < row_end && row_ok[b * 128 + t] != 0;
-      // logits in log2 units; x is reused for the max reduction and the probabilities
-      float x[32];
-      {
-        uint32_t sr[32];
-        tmem_ld16(s_addr, sr);
-        tmem_ld16(s_addr + 16, sr + 16);
-        tmem_wait_ld();
+      tmem_wait_ld();
+      // d = logit (log2 units) - running max of its head; -inf for a row without a key
+      float d[32];
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        const float4 hs = *reinterpret_cast<const float4*>(hscale + h0 + i);
+        const float4 mm = *reinterpret_cast<const float4*>(m_run + h0 + i);
+        d[i] = valid ? fmaf(__uint_as_float(sr[i]), hs.x, -mm.x) : -INFINITY;
+        d[i + 1] = valid ? fmaf(__uint_as_float(sr[i + 1]), hs.y, -mm.y) : -INFINITY;
+        d[i + 2] = valid ? fmaf(__uint_as_float(sr[i + 2]), hs.z, -mm.z) : -INFINITY;
+        d[i + 3] = valid ? fmaf(__uint_as_float(sr[i + 3]), hs.w, -mm.w) : -INFINITY;
+      }
+      bool over = false;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) over |= d[i] > kRescaleThreshold;
+      const bool move_max = named_bar_or(1, 256, over);  // always true on the first tile with a valid row
+      if (move_max) {
+        float x[32];  // the logits themselves, for the new maxima
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           const float4 hs = *reinterpret_cast<const float4*>(hscale + h0 + i);
@@ -669,19 +681,7 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
           x[i + 2] = valid ? __uint_as_float(sr[i + 2]) * hs.z : -INFINITY;
           x[i + 3] = valid ? __uint_as_float(sr[i + 3]) * hs.w : -INFINITY;
         }
-      }
-      bool over = false;
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        const float4 mm = *reinterpret_cast<const float4*>(m_run + h0 + i);
-        over |= x[i] > mm.x + kRescaleThreshold;
-        over |= x[i + 1] > mm.y + kRescaleThreshold;
-        over |= x[i + 2] > mm.z + kRescaleThreshold;
-        over |= x[i + 3] > mm.w + kRescaleThreshold;
-      }
-      const bool move_max = named_bar_or(1, 256, over);  // always true on the first tile with a valid row
-      if (move_max) {
-        xreduce32<true>(x);  // x[0] = this warp's max of head h0 + lane (x is reloaded below)
+        xreduce32<true>(x);  // x[0] = this warp's max of head h0 + lane
         red_max[q4 * 64 + h0 + lane] = x[0];
         named_bar_sync(1, 256);
         if (threadIdx.x < kH) {
@@ -695,33 +695,25 @@ __device__ __forceinline__ void attend(const AttnParams& p, const CUtensorMap& t
         named_bar_sync(1, 256);
 #pragma unroll
         for (int i = 0; i < 32; ++i) lacc[i] *= alpha[h0 + i];
-        uint32_t sr[32];  // S^T[b] is intact until s_free[b] is arrived on below
-        tmem_ld16(s_addr, sr);
-        tmem_ld16(s_addr + 16, sr + 16);
-        tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           const float4 hs = *reinterpret_cast<const float4*>(hscale + h0 + i);
-          x[i] = valid ? __uint_as_float(sr[i]) * hs.x : -INFINITY;
-          x[i + 1] = valid ? __uint_as_float(sr[i + 1]) * hs.y : -INFINITY;
-          x[i + 2] = valid ? __uint_as_float(sr[i + 2]) * hs.z : -INFINITY;
-          x[i + 3] = valid ? __uint_as_float(sr[i + 3]) * hs.w : -INFINITY;
+          const float4 mm = *reinterpret_cast<const float4*>(m_run + h0 + i);
+          d[i] = valid ? fmaf(__uint_as_float(sr[i]), hs.x, -mm.x) : -INFINITY;
+          d[i + 1] = valid ? fmaf(__uint_as_float(sr[i + 1]), hs.y, -mm.y) : -INFINITY;
+          d[i + 2] = valid ? fmaf(__uint_as_float(sr[i + 2]), hs.z, -mm.z) : -INFINITY;
+          d[i + 3] = valid ? fmaf(__uint_as_float(sr[i + 3]), hs.w, -mm.w) : -INFINITY;
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[b]);  // QK of tile it + 2 may overwrite S^T[b]
+      float pr[32];  // probabilities 2^d (2^-inf = 0)
 #pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        const float4 mm = *reinterpret_cast<const float4*>(m_run + h0 + i);
-        x[i] = valid ? fast_exp2(x[i] - mm.x) : 0.f;
-        x[i + 1] = valid ? fast_exp2(x[i + 1] - mm.y) : 0.f;
-        x[i + 2] = valid ? fast_exp2(x[i + 2] - mm.z) : 0.f;
-        x[i + 3] = valid ? fast_exp2(x[i + 3] - mm.w) : 0.f;
+      for (int i = 0; i < 32; ++i) {
+        pr[i] = fast_exp2(d[i]);
+        lacc[i] += pr[i];
       }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) lacc[i] += x[i];
-      float (&pr)[32] = x;
       // P[b] was last read by PV of tile it - 2, which completed before QK of this tile
       // signalled s_full (one thread issues both, and a commit covers every earlier MMA)
       // P in the third buffer, last read by PV of tile it - 1, which completed before QK of
