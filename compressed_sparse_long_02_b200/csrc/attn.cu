@@ -81,9 +81,7 @@ constexpr uint32_t kColO2 = 256;    // two-pass: S^T of up to 3 tiles in [0, 192
 // (free once the last QK has completed).  Barrier pairs: K slot s and V slot s < kRing
 // share pair s; V slot kRing + i uses pair kRing + kPBufs + i.
 constexpr int kSlotsK2 = kRing + kPBufs;
-constexpr int kSlotsV2 = kRing + 4;
 constexpr int kSlotBars = kRing + kPBufs + 4;
-static_assert(kSlotsV2 % 2 == 0, "V slabs go in adjacent pairs");
 constexpr size_t kOffQ = 0;                                       // 64 KB: [8 d-atoms][64 heads][128 B]
 constexpr size_t kOffRing = 64 * 1024;                            // kRing x 16 KB
 constexpr size_t kOffP = kOffRing + kRing * kSlabBytes;           // kPBufs x 16 KB: [128 keys][128 B]
@@ -835,29 +833,64 @@ __device__ __forceinline__ Slot2 slot_k2(int j) {
   r.parity = static_cast<uint32_t>(j / kSlotsK2) & 1u;
   return r;
 }
-__device__ __forceinline__ Slot2 slot_v2(int v, int nK) {
-  const int sl = v % kSlotsV2;
-  Slot2 r;
-  if (sl < kRing) {
+
+// The V pass takes the share's tiles in the order vtile(0), vtile(1), ..., a 128-dim chunk
+// (two adjacent 16 KB slots) at a time.  With one or three tiles ("resident" plan), three
+// chunks of the last K tile are still in the ring when the K pass ends, each in one of
+// the ring's slot pairs (0,1), (2,3), (4,5) (chunks 1-3 of tile 2, chunks 0-2 of tile 0):
+// that tile goes first and those chunks are not gathered again; every other chunk is
+// gathered into the next slot pair of a cycle of five -- the two pairs of Q's slots
+// (free after the last QK) first under the resident plan, the ring's pairs first
+// otherwise.
+__device__ __forceinline__ bool v_resident_plan(int n_tiles) { return n_tiles == 1 || n_tiles == 3; }
+__device__ __forceinline__ int vtile(int i, int n_tiles) {
+  return v_resident_plan(n_tiles) ? (i == 0 ? n_tiles - 1 : i - 1) : i;
+}
+// The ring pair holding chunk dc of the first V tile after the K pass, or -1 (gathered).
+__device__ __forceinline__ int v_resident_pair(int dc, int n_tiles) {
+  if (!v_resident_plan(n_tiles)) return -1;
+  const int sl = ((n_tiles - 1) * kSlabs + 2 * dc) % kSlotsK2;  // slot_k2 of the chunk's first slab
+  return (sl % 2 == 0 && sl + 1 < kRing) ? sl / 2 : -1;
+}
+struct VPair {
+  uint32_t off;    // the first slot's offset (the second follows it)
+  int bar;         // the first slot's barriers (the second: bar + 1)
+  uint32_t free_parity, full_parity;
+  bool q_slots;    // the pair is two of Q's slots
+};
+// Slots and barrier phases of the g-th gathered chunk of the V pass.  A pair's uses of
+// slot_free: its K-pass uses, the resident chunk (resident plan, ring pairs), then earlier
+// gathered chunks; its uses of full: the same without the resident chunk (never loaded).
+__device__ __forceinline__ VPair v_pair(int g, int nK, int n_tiles) {
+  const bool res = v_resident_plan(n_tiles);
+  const int c = g % 5, prev = g / 5;
+  const int ring = res ? c - 2 : c;  // ring pair index, or negative / >= 3 for Q's pairs
+  VPair r;
+  if (ring >= 0 && ring < 3) {
+    const int sl = 2 * ring;
     const int k_uses = nK > sl ? (nK - 1 - sl) / kSlotsK2 + 1 : 0;  // K slabs that used this pair
     r.off = static_cast<uint32_t>(kOffRing + sl * kSlabBytes);
     r.bar = sl;
-    r.parity = static_cast<uint32_t>(k_uses + v / kSlotsV2) & 1u;
+    r.free_parity = static_cast<uint32_t>(k_uses + (res ? 1 : 0) + prev) & 1u;
+    r.full_parity = static_cast<uint32_t>(k_uses + prev) & 1u;
+    r.q_slots = false;
   } else {
-    r.off = static_cast<uint32_t>(kOffQ + (sl - kRing) * kSlabBytes);
-    r.bar = kRing + kPBufs + (sl - kRing);
-    r.parity = static_cast<uint32_t>(v / kSlotsV2) & 1u;
+    const int q = 2 * (res ? c : c - 3);  // Q's slot pair (q, q + 1)
+    r.off = static_cast<uint32_t>(kOffQ + q * kSlabBytes);
+    r.bar = kRing + kPBufs + q;
+    r.free_parity = r.full_parity = static_cast<uint32_t>(prev) & 1u;
+    r.q_slots = true;
   }
   return r;
 }
 
 // Two-pass variant for a share of at most kMaxTiles2 tiles (decode: a query split over
-// several CTAs).  Slab order K0 | K1 | ... | K(n-1) | V0 | ... | V(n-1): the K pass is a
-// pure stream from HBM that QK consumes as slabs land (S^T of tile t in TMEM columns
-// 64 t), independent of the softmax; the softmax then runs once over every tile with
-// the exact maximum (no rescaling of O^T); the V pass re-gathers the same rows, now in
-// L2, into the ring slots the K pass frees, while the softmax works, and PV accumulates
-// O^T in columns [256, 512).  Same outputs as attend(): the normalised result or the
+// several CTAs).  The K pass is a pure stream from HBM that QK consumes as slabs land
+// (S^T of tile t in TMEM columns 64 t), independent of the softmax; the softmax then runs
+// once over every tile with the exact maximum (no rescaling of O^T); the V pass takes the
+// rows again, tile by tile in the order vtile(), re-gathering them from L2 into slots
+// that are free (or still finding them in the ring: the resident chunks of the last K
+// tile), and PV accumulates O^T in columns [256, 512).  Same outputs as attend(): the normalised result or the
 // unnormalised partial with its (max, sum).
 __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensorMap& tm_q, const CUtensorMap& tm_e,
                                              const CUtensorMap& tm_w, uint8_t* smem, uint32_t tmem, int n,
@@ -886,36 +919,56 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
     __syncwarp();
     bool ok = true;
     const int nK = kSlabs * n_tiles;
-    bool q_free = false;  // the last QK has completed: Q's slabs may take V slabs
-    for (int st = 0; ok && st < 2 * n_tiles; ++st) {
-      const bool is_v = st >= n_tiles;
-      const int tile = is_v ? st - n_tiles : st;
+    // K pass: tile t's slab ka is slab j = 8 t + ka of the K ring
+    for (int tile = 0; ok && tile < n_tiles; ++tile) {
       const uint16_t* src_row = key_row_src(p, kl, n, row_begin + tile * kBN + my_row, row_begin, row_end,
-                                            staged ? L.sidx : nullptr, !is_v);
+                                            staged ? L.sidx : nullptr, true);
       const bool valid = src_row != nullptr;
       const unsigned long long src_ll = reinterpret_cast<unsigned long long>(valid ? src_row : p.entries);
       const TileBox box = tile_box(p, kl, tm_e, tm_w, row_begin + tile * kBN, row_end);
-      if (ptid == 0) CSA_T(tslot, 8 + st);
-      if (!is_v) {  // published before this tile's first slab is issued
-        L.row_ok[tile * 128 + my_row] = valid ? 1 : 0;
-        mbar_arrive(&L.row_ready[tile]);
-      }
+      if (ptid == 0) CSA_T(tslot, 8 + tile);
+      L.row_ok[tile * 128 + my_row] = valid ? 1 : 0;  // published before the tile's first slab is issued
+      mbar_arrive(&L.row_ready[tile]);
       for (int ka = 0; ka < kSlabs; ++ka) {
-        const int j = is_v ? nK + tile * kSlabs + ka : tile * kSlabs + ka;  // slab sequence number
-        const Slot2 sl = is_v ? slot_v2(j - nK, nK) : slot_k2(j);
-        if (is_v && sl.bar >= kRing + kPBufs && !q_free) {
-          if (!warp_wait(&L.s_full[n_tiles - 1], 0, p.err, L.abort_flag)) {
-            ok = false;
-            break;
-          }
-          q_free = true;
-        }
+        const int j = tile * kSlabs + ka;
+        const Slot2 sl = slot_k2(j);
         if (!warp_wait(&L.slot_free[sl.bar], sl.parity ^ 1, p.err, L.abort_flag)) {
           ok = false;
           break;
         }
         if (ptid == 0 && tslot == 4 && j < 64) CSA_T(10, j);
         gather_slab(smem_u32(smem + sl.off), box, ka, src_ll, valid, pw, lane, &L.full[sl.bar]);
+      }
+    }
+    // V pass: the same rows again (now in L2), chunk by chunk, except the resident chunks
+    bool q_free = false;  // the last QK has completed: Q's slots may take V slabs
+    int g = 0;            // gathered chunks so far
+    for (int vi = 0; ok && vi < n_tiles; ++vi) {
+      const int tile = vtile(vi, n_tiles);
+      const uint16_t* src_row = key_row_src(p, kl, n, row_begin + tile * kBN + my_row, row_begin, row_end,
+                                            staged ? L.sidx : nullptr, false);
+      const bool valid = src_row != nullptr;
+      const unsigned long long src_ll = reinterpret_cast<unsigned long long>(valid ? src_row : p.entries);
+      const TileBox box = tile_box(p, kl, tm_e, tm_w, row_begin + tile * kBN, row_end);
+      if (ptid == 0) CSA_T(tslot, 8 + n_tiles + vi);
+      for (int dc = 0; ok && dc < 4; ++dc) {
+        if (vi == 0 && v_resident_pair(dc, n_tiles) >= 0) continue;  // still in the ring
+        const VPair vp = v_pair(g++, nK, n_tiles);
+        if (vp.q_slots && !q_free) {
+          if (!warp_wait(&L.s_full[n_tiles - 1], 0, p.err, L.abort_flag)) {
+            ok = false;
+            break;
+          }
+          q_free = true;
+        }
+        for (int h = 0; h < 2; ++h) {
+          if (!warp_wait(&L.slot_free[vp.bar + h], vp.free_parity ^ 1, p.err, L.abort_flag)) {
+            ok = false;
+            break;
+          }
+          gather_slab(smem_u32(smem + vp.off + h * kSlabBytes), box, 2 * dc + h, src_ll, valid, pw, lane,
+                      &L.full[vp.bar + h]);
+        }
       }
     }
     cp_async_wait_all();
@@ -967,37 +1020,49 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
       }
       __syncwarp();
     }
-    // V pass: O^T += V^T P^T[tile], a 128-dim chunk (two adjacent slots) at a time; tile t
-    // starts as soon as its P is written (the softmax publishes P tile by tile)
+    // V pass: O^T += V^T P^T[tile], a 128-dim chunk (two adjacent slots) at a time, tiles in
+    // the order vtile(0), vtile(1), ...; a tile starts as soon as its P is written (the
+    // softmax publishes P tile by tile, in the same order); resident chunks need no wait
     if (lane == 0) CSA_T(tslot, 30);
-    for (int tile = 0; ok && tile < n_tiles; ++tile) {
+    int g = 0;  // gathered chunks so far
+    for (int vi = 0; ok && vi < n_tiles; ++vi) {
+      const int tile = vtile(vi, n_tiles);
       if (!warp_wait(&L.row_ready[tile], 1, p.err, L.abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
       for (int dc = 0; dc < 4; ++dc) {
-        const int v = tile * kSlabs + 2 * dc;  // even: the chunk's two slabs sit in adjacent slots
-        const Slot2 s0 = slot_v2(v, nK), s1 = slot_v2(v + 1, nK);
-        if (!warp_wait(&L.full[s0.bar], s0.parity, p.err, L.abort_flag) ||
-            !warp_wait(&L.full[s1.bar], s1.parity, p.err, L.abort_flag)) {
-          ok = false;
-          break;
+        const int rp = vi == 0 ? v_resident_pair(dc, n_tiles) : -1;
+        uint32_t off;
+        int bar;
+        if (rp >= 0) {  // the K pass's slabs, still in ring slots 2 rp, 2 rp + 1
+          off = static_cast<uint32_t>(kOffRing + 2 * rp * kSlabBytes);
+          bar = 2 * rp;
+        } else {
+          const VPair vp = v_pair(g++, nK, n_tiles);
+          if (!warp_wait(&L.full[vp.bar], vp.full_parity, p.err, L.abort_flag) ||
+              !warp_wait(&L.full[vp.bar + 1], vp.full_parity, p.err, L.abort_flag)) {
+            ok = false;
+            break;
+          }
+          off = vp.off;
+          bar = vp.bar;
         }
         fence_proxy_async_smem();
         tc_fence_after();
         if (lane == 0) {
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_bf16(tmem + kColO2 + 64 * dc, smem_desc(base + s0.off + ks * 2048, kSlabBytes, 1024, kSwizzle128B),
+            mma_bf16(tmem + kColO2 + 64 * dc, smem_desc(base + off + ks * 2048, kSlabBytes, 1024, kSwizzle128B),
                      smem_desc(p0 + tile * 16384 + ks * 2048, 16384, 1024, kSwizzle128B), idesc_pv,
-                     (tile > 0 || ks > 0) ? 1u : 0u);
-          tc_commit(&L.slot_free[s0.bar]);
-          tc_commit(&L.slot_free[s1.bar]);
+                     (vi > 0 || ks > 0) ? 1u : 0u);
+          tc_commit(&L.slot_free[bar]);
+          tc_commit(&L.slot_free[bar + 1]);
         }
         __syncwarp();
       }
-      if (lane == 0) CSA_T(tslot, 32 + tile);
+      if (lane == 0) CSA_T(tslot, 32 + vi);
     }
     if (ok && lane == 0) tc_commit(L.fin);
     __syncwarp();
@@ -1055,11 +1120,13 @@ __device__ __forceinline__ void attend_2pass(const AttnParams& p, const CUtensor
       }
       named_bar_sync(1, 256);
     }
-    // sweep 2: P = 2^(x - max) as bf16 per tile, and the per-thread sums
+    // sweep 2: P = 2^(x - max) as bf16 per tile, and the per-thread sums, tiles in the V
+    // pass's order
     float lacc[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) lacc[i] = 0.f;
-    for (int it = 0; ok && it < n_tiles; ++it) {
+    for (int vi = 0; ok && vi < n_tiles; ++vi) {
+      const int it = vtile(vi, n_tiles);
       const bool valid = row_begin + it * kBN + t < row_end && L.row_ok[it * 128 + t] != 0;
       float x[32];
       uint32_t sr[32];
