@@ -91,8 +91,8 @@ def measure_tensor_peaks(dev, reps: int = 3) -> dict:
 # decode step (profiles/*_decode_128k.md), keyed by the sha1 of the kernel's source file
 # at capture time: a kernel changed since its capture reports traffic null.
 NCU_TRAFFIC = {
-    "attention": {"bytes": 40103680 + 720640, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
-                  "sha1": "fef08f8a7e38d7502b3cfb83dd239ab69d7d0434"},
+    "attention": {"bytes": 40066048 + 717312, "src": "compressed_sparse_long_02_b200/csrc/attn.cu",
+                  "sha1": "4559cbf1e5cbfa46e50cc43a5a7a30025fa7a6fa"},
     "index_score": {"bytes": 71483904 + 1665792, "src": "compressed_sparse_long_02_b200/csrc/index.cu",
                     "sha1": "b271de5f29ab6b90adcc34a460af7ad5b475c231"},
     "topk_select": {"bytes": 4253184, "src": "compressed_sparse_long_02_b200/csrc/topk.cu",
