@@ -142,3 +142,42 @@ def test_index_fusion_switch_plan(L):
         assert B.csa_index_topk_launches(0, 64, 128, 32768, 1024) == 0
     finally:
         B.csa_set_index_fusion(False)
+
+
+def test_validation_of_the_newer_calls(L):
+    """The multi-query indexer, the attention calls that prepare raw queries, and the grouped
+    output projection reject what they do not support with a status, before any device
+    work (null pointers past the checks stop at INVALID_ARG, never at a launch)."""
+    from compressed_sparse_long_02_b200 import binding as B
+    P = ctypes.c_void_p
+    x = P(16)
+    ws = 1 << 30
+
+    def grouped(q_group, Nq, Hi, Di, E_max=64):
+        return L.csa_index_topk_grouped(q_group, Nq, Hi, Di, 8, 4, x, x, x, x, x, 1, E_max, x, x, x, x, x, None, x, ws,
+                                        None)
+
+    assert grouped(3, 2, 64, 128) == 3     # only one or two query rows per group
+    assert grouped(2, 2, 32, 128) == 3     # groups of two need 64 heads of 128 dims
+    assert grouped(2, 2, 64, 64) == 3
+    assert grouped(2, 2, 64, 128, E_max=60) == 3
+    assert grouped(2, 0, 64, 128) == 0     # nothing to do
+    assert L.csa_index_topk_grouped(2, 2, 64, 128, 8, 4, *([None] * 5), 1, 64, *([None] * 5), None, None, ws,
+                                    None) == 1
+
+    def attn_ex(rope_dims, eps=1e-6, theta=1e4, norm=1):
+        prep = ctypes.byref(B._QPrep(norm, eps, rope_dims, theta))
+        return L.csa_sparse_attn_ex(prep, 1, 64, 512, 8, 128, ctypes.c_float(0.04), x, x, x, 1, 64, x, x, x, 128, x, x,
+                                    x, None, x, ws, None)
+
+    for rd in (66, 3, -2):                 # RoPE on 0..64 even channels only
+        assert attn_ex(rd) == 3
+    assert attn_ex(64, eps=-1.0) == 1      # a negative epsilon
+    assert attn_ex(64, theta=0.0) == 1     # RoPE without a base
+    prep = ctypes.byref(B._QPrep(1, 1e-6, 66, 1e4))
+    assert L.hca_attn_ex(prep, 1, 64, 512, 128, 128, ctypes.c_float(0.04), x, x, x, 1, 64, x, x, 128, x, x, x, None,
+                         x, ws, None) == 3
+    # grouped output projection: heads split evenly over groups, tile-friendly sizes
+    assert L.csa_grouped_out_proj(16, 64, 512, 7, 1024, 4096, x, x, x, x, x, None) == 1
+    assert L.csa_grouped_out_proj(16, 64, 512, 8, 1000, 4096, x, x, x, x, x, None) == 3
+    assert L.csa_grouped_out_proj(16, 64, 512, 8, 1024, 4000, x, x, x, x, x, None) == 3
